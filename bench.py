@@ -1,0 +1,359 @@
+"""Benchmark of the tiled distance-map sampler's hot path.
+
+One step = one pass of the whole path over one batch: the fused DDIM run (init
+noise, stand-in eps of both streams, guidance, update, overlap projection after
+every step) on a 32-tile chain x 1000 samples (w = 1, 50 steps), classical-MDS
+recovery of all 32,000 maps, distance reconstruction and the seam discrepancy
+(Eq. 6 of the ParaChromo paper) of the reconstructed maps.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Under torchrun every rank runs its own 1000 samples of a joint N*1000-sample
+run (weak scaling); the only collective is one all-reduce of the per-seam
+overlap sums that Eq. (6) averages over all samples.  Rank 0 prints one JSON
+line.  ``--impl reference`` times the float64 CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = synth.WORKLOADS["chain32_b1000_cfg"]
+METRIC = "map-denoise-steps/sec (64-bead fp32 maps) on 1 B200; % FP32/HBM roofline"
+UNIT = "map-steps/s"
+
+# Algorithmic operations of one quad-step of the fused run (one 4-entry row
+# quad of the folded state advanced one DDIM step), counted per lane:
+#   Philox4x32-10 call: 10 rounds x (2 mul.wide + 4 xor + 2 key adds) + 3 counter ops = 83
+#   Box-Muller pair: 2 shifts, 1 add, 2 int->float, 2 scales, log, mul, sqrt,
+#                    mul, sincospi, 2 muls = 15
+#   one noise stream per quad: 83 + 2 x 15 = 113
+#   update: one FMA per entry per term (x_t, x0, each noise stream)
+OPS_PHILOX = 83
+OPS_BOX_MULLER_PAIR = 15
+QUADS_PER_MAP = 544
+
+
+def ops_per_map_step(n_streams: int) -> int:
+    per_quad = n_streams * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR) + 4 * (2 + n_streams)
+    return QUADS_PER_MAP * per_quad
+
+
+def alu_peak_ops(sms: int = 148, clock_ghz: float = 1.965) -> float:
+    """Issue ceiling: one lane-op per CUDA-core lane per clock (128 per SM)."""
+    return sms * 128 * clock_ghz * 1e9
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not sampled"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---- the oracle arm ---------------------------------------------------------------
+
+def oracle_sample(b_count: int = 2, mds_maps: int = 8):
+    """One bounded sample of the workload on the CPU oracle: the full run of
+    ``b_count`` joint samples (all 32 tiles, 50 steps), classical MDS and
+    reconstruction of ``mds_maps`` of their maps (the recovery time is scaled
+    to all maps of the sample: maps are independent) and Eq. (6).
+    Returns (seconds, map-steps)."""
+    from oracle import mds as omds, schedule as osched, seam as oseam
+    from oracle.ddim import ddim_run
+    wl = WORKLOAD
+    x0 = synth.chain_x0(wl.seed, 1, wl.T, sigma=wl.sigma)
+    t0 = time.perf_counter()
+    sch = osched.Schedule(S=wl.S, eta=wl.eta)
+    out = ddim_run(x0, sch, wl.w, wl.s_c, wl.s_u, wl.seed, np.arange(b_count), wl.B)
+    t1 = time.perf_counter()
+    flat = out.reshape(-1, 64, 64)
+    X, _ = omds.classical_mds(flat[:mds_maps])
+    omds.pairwise_distances(X)
+    t2 = time.perf_counter()
+    oseam.seam_discrepancy(out)
+    t3 = time.perf_counter()
+    total = (t1 - t0) + (t2 - t1) * flat.shape[0] / mds_maps + (t3 - t2)
+    return total, b_count * wl.T * wl.S
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except ImportError:
+        pass
+    times, steps = [], 0
+    for i in range(args.warmup + args.steps):
+        dt, ms = oracle_sample()
+        if i >= args.warmup:
+            times.append(dt)
+            steps = ms
+    t_step = float(np.mean(times))
+    value = steps / t_step
+    sample = ("per step: 2 joint samples x 32 tiles x 50 steps (3,200 map-steps) of the 32-tile chain, "
+              "classical MDS + reconstruction timed on 8 of their 64 maps and scaled to 64, Eq. 6; "
+              "single-threaded float64 numpy")
+    cpu = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(world),
+            "cpu_baseline": cpu, "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(world):
+    wl = WORKLOAD
+    return {"workload": "chain32_b1000_cfg: 1 chain x 32 tiles x 1000 samples per GPU, 12-bead overlaps, "
+                        "DDIM 50 steps eta 0, CFG w=1 (eps_c 0.1, eps_u 0.3), projection every step, "
+                        "then MDS + reconstruction + seam discrepancy",
+            "C": wl.C, "T": wl.T, "B_per_gpu": wl.B, "S": wl.S, "maps_per_gpu": wl.n_maps,
+            "parallelism": f"samples sharded over {world} GPU(s)",
+            "l2": "working set 1.1 GB per GPU > 126 MB L2; no flush"}
+
+
+# ---- our arm ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import tiled_distance_maps_b200 as tdm
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOAD
+    B, T, S = wl.B, wl.T, wl.S
+    n_maps = wl.n_maps
+    tiling = tdm.Tiling(C=1, T=T, B=B, overlap=wl.overlap, sync_every=wl.sync_every,
+                        B_total=B * world, b_offset=B * rank)
+    ctx = tdm.context(local_rank)
+    sched = tdm.Schedule(S, wl.eta, ctx=ctx)
+    x0_host = torch.from_numpy(synth.chain_x0(wl.seed, 1, T, sigma=wl.sigma)).contiguous()
+    x0 = x0_host.to(dev)
+    maps = torch.empty(n_maps * 4096, device=dev)
+    coords = torch.empty(n_maps * 192, device=dev)
+    eig = torch.empty(n_maps * 3, device=dev)
+    rec = torch.empty(n_maps * 4096, device=dev)
+    sums = torch.empty((T - 1) * wl.overlap ** 2, device=dev)
+    disc = torch.empty(T - 1, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev_run = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)]
+
+    def step(i_timed=None):
+        if i_timed is not None:
+            ev_run[2 * i_timed].record(stream)
+        tdm.ddim_run(sched, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, tiling, ctx=ctx)
+        if i_timed is not None:
+            ev_run[2 * i_timed + 1].record(stream)
+        tdm.mds_recover(maps, n_maps, coords, eig, ctx=ctx)
+        tdm.pairwise_dist(coords, n_maps, rec, ctx=ctx)
+        tdm.seam_overlap_sums(rec, tiling, sums, ctx=ctx)
+        if world > 1:
+            torch.distributed.all_reduce(sums)
+        tdm.seam_discrepancy_finalize(sums, tiling, disc, ctx=ctx)
+
+    launches_per_step = 1 + 1 + 1 + (2 if _seam_chunks(T - 1, B) > 1 else 1) + 1
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flags = tdm.ctx_sync(ctx)
+
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(args.steps):
+            step(i)
+        stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = start.elapsed_time(stop)
+    run_ms = [ev_run[2 * i].elapsed_time(ev_run[2 * i + 1]) for i in range(args.steps)]
+    flags |= tdm.ctx_sync(ctx)
+
+    # end to end through the public API from host buffers
+    pinned_x0 = x0_host.pin_memory()
+    h_coords = torch.empty(n_maps * 192, dtype=torch.float32).pin_memory()
+    h_eig = torch.empty(n_maps * 3, dtype=torch.float32).pin_memory()
+    h_disc = torch.empty(T - 1, dtype=torch.float32).pin_memory()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        x0.copy_(pinned_x0, non_blocking=True)
+        step()
+        h_coords.copy_(coords, non_blocking=True)
+        h_eig.copy_(eig, non_blocking=True)
+        h_disc.copy_(disc, non_blocking=True)
+    e_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_stop)
+
+    t = torch.tensor([ms, e2e_ms, float(np.mean(run_ms))], device=dev, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms, e2e_ms, run_avg_ms = t.tolist()
+
+    if rank == 0:
+        map_steps = world * n_maps * S
+        value = map_steps * args.steps / (ms / 1e3)
+        peaks, kind = measured_peaks()
+        clk = clocks.summary()
+        n_streams = (1 if wl.w == 0 else 2) + (1 if wl.eta > 0 else 0)
+        ops = ops_per_map_step(n_streams) * n_maps * S + QUADS_PER_MAP * n_maps * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR)
+        achieved = ops / (run_avg_ms / 1e3)
+        peak = alu_peak_ops(148, float(peaks.get("sm_max_mhz", 1965.0)) / 1e3)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": _config(world),
+            "roofline": {"kernel": "ddim_run_kernel", "bound": "alu", "achieved": achieved / 1e12,
+                         "peak": peak / 1e12, "unit": "Tops/s", "frac": achieved / peak, "traffic": None,
+                         "peak_kind": "derived: 148 SMs x 128 lanes x max SM clock",
+                         "ms_per_launch": run_avg_ms,
+                         "ops_per_launch": ops},
+            "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
+            "e2e": {"value": map_steps * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": x0_host.numel() * 4,
+                    "d2h_bytes_per_step": (n_maps * 195 + (T - 1)) * 4},
+            "gpu_launches": launches_per_step * args.steps,
+            "mds_not_converged": bool(flags & tdm.FLAG_MDS_NOT_CONVERGED),
+            "peaks": kind,
+        }
+        if args.cpu_baseline and world == 1:
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(1):
+                    dt, msteps = oracle_sample(4, 16)
+            except ImportError:
+                dt, msteps = oracle_sample(4, 16)
+            line["cpu_baseline"] = {"value": msteps / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": "4 joint samples x 32 tiles x 50 steps (6,400 map-steps) of the "
+                                              "32-tile chain, classical MDS + reconstruction timed on 16 of "
+                                              "their 128 maps and scaled to 128, Eq. 6; single-threaded "
+                                              "float64 numpy"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def _seam_chunks(n_seams, B):
+    target = 4 * 148
+    if n_seams >= target // 2 or B <= 8:
+        return 1
+    ch = -(-target // n_seams)
+    return max(1, min(ch, -(-B // 8)))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,219 @@
+/*
+ * tdm.h -- C ABI of the tiled distance-map sampler library (libtdm.so), sm_100a.
+ *
+ * The library implements the data-parallel hot path of a ParaChromo-style tiled
+ * 3D-genome diffusion sampler (ParaChromo paper, mdpi.com/2079-9292/15/13/2750):
+ * batched DDIM reverse updates on 64-bead distance maps with classifier-free
+ * guidance, the overlap-consistency projection of the 12-bead seam between
+ * adjacent tiles (§4.3.2, Algorithm 1), coordinate recovery by classical MDS
+ * (the distance-geometry initialisation of §3.1), pairwise-distance
+ * reconstruction and the seam discrepancy of §5.5 Eq. (6).  The trained U-Net
+ * is replaced by a stand-in noise predictor: the ideal denoiser toward a known
+ * x0 plus counter-based Philox noise.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every function returns a tdm_status; TDM_OK is 0.  Argument errors are
+ *    found before any launch and return TDM_EINVAL / TDM_EUNSUPPORTED without
+ *    touching device memory.  tdm_ctx_last_error() gives a one-line detail.
+ *  - Compute entry points are asynchronous on the caller's stream (a
+ *    cudaStream_t passed as tdm_stream; NULL is the legacy default stream).
+ *    Launch failures are reported as TDM_ECUDA.
+ *  - Every pointer named "device" is device memory owned by the caller; it must
+ *    be 16-byte aligned and hold contiguous row-major float32 data.  The library
+ *    never frees caller memory and allocates only inside tdm_ctx_create,
+ *    tdm_init_schedule and on the first use of a new tiling shape (a small
+ *    lookup table, cached in the context).
+ *  - Beads per tile n is 64.  A map is 64 x 64 float32 (16 KiB).
+ *  - Tiled maps are laid out [C][T][B][64][64]: chain c, tile k, sample b.
+ *    Reference maps x0 are [C][T][64][64], shared by the B samples of a tile
+ *    (§3.3: samples of one condition differ only through their noise).
+ *  - The noise id of map (c, k, b) is
+ *        g = sample_id_base + (c*T + k) * B_total + b_offset + b
+ *    so a run split into sample shards or chunks reproduces the unsplit run.
+ */
+#ifndef TDM_H
+#define TDM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t tdm_status;
+#define TDM_OK             0
+#define TDM_EINVAL         1  /* bad argument (null, misaligned, out of range) */
+#define TDM_ECUDA          2  /* a CUDA runtime call or launch failed */
+#define TDM_ETIMEOUT       3  /* reserved: no kernel of this library waits on another */
+#define TDM_ENONFINITE     4  /* reserved for a non-finite scan of outputs */
+#define TDM_EUNSUPPORTED   5  /* valid request this build does not implement */
+#define TDM_ENOMEM         6  /* device allocation failed */
+#define TDM_ENOTCONVERGED  7  /* an MDS eigen-solve hit its iteration cap (see tdm_ctx_sync) */
+
+/* noise streams of the stand-in and the sampler (Philox counter word 3, top byte) */
+#define TDM_STREAM_INIT   0  /* initial state x_T */
+#define TDM_STREAM_EPS_C  1  /* conditional eps stream */
+#define TDM_STREAM_EPS_U  2  /* unconditional eps stream */
+#define TDM_STREAM_ETA    3  /* sigma_i z of DDIM with eta > 0 */
+
+/* device status flags returned by tdm_ctx_sync */
+#define TDM_FLAG_MDS_NOT_CONVERGED 0x1u
+
+/* columns of the host schedule table (tdm_schedule_table), one row per DDIM step i */
+#define TDM_SCHED_COLS 8   /* tau_i, ab_t, ab_p, sigma_i, a_i, b_i, sqrt(ab_t), 1/sqrt(1-ab_t) */
+
+typedef void *tdm_stream;              /* a cudaStream_t */
+typedef struct tdm_ctx tdm_ctx;        /* opaque: device, status word, scratch, plan cache */
+typedef struct tdm_schedule tdm_schedule;  /* opaque: DDIM coefficient table */
+
+/* Shape of a tiled batch.  C chains of T tiles (T = 1: independent, untiled
+ * maps), B samples per tile in this call; adjacent tiles share `overlap` beads
+ * (12 in ParaChromo §3.2).  The projection runs after every `sync_every`-th
+ * DDIM step counted from the start (0: never).  B_total (0 means B) is the
+ * number of samples of the whole run when this call holds the slice
+ * [b_offset, b_offset + B) of them; sample_id_base offsets every noise id. */
+typedef struct tdm_tiling {
+    int32_t C;
+    int32_t T;
+    int32_t B;
+    int32_t overlap;
+    int32_t sync_every;
+    int32_t reserved;     /* must be 0 */
+    int64_t B_total;
+    int64_t b_offset;
+    int64_t sample_id_base;
+} tdm_tiling;
+
+/* ---- context ---------------------------------------------------------- */
+
+/* Creates a context on CUDA device `device` (allocates its status word and
+ * scratch).  *out receives the handle.  Errors: TDM_EINVAL (out NULL or bad
+ * device), TDM_ENOMEM, TDM_ECUDA. */
+tdm_status tdm_ctx_create(tdm_ctx **out, int32_t device);
+
+/* Frees everything the context owns.  NULL is ignored. */
+void tdm_ctx_destroy(tdm_ctx *ctx);
+
+/* Static message for a status code (never NULL). */
+const char *tdm_status_str(tdm_status s);
+
+/* Detail of the last error seen on this context ("" if none). */
+const char *tdm_ctx_last_error(const tdm_ctx *ctx);
+
+/* Synchronises `stream`, then reads and clears the context's device status
+ * word.  *flags_out (may be NULL) receives the TDM_FLAG_* bits raised since the
+ * last call.  Returns TDM_ENOTCONVERGED when TDM_FLAG_MDS_NOT_CONVERGED was set. */
+tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out);
+
+/* ---- schedule (ParaChromo §4.1, §5.1.1: reduced-step DDIM) --------------
+ * Builds, in float64 on the host, beta_t linear from beta_start to beta_end
+ * over T_train steps (or takes alphas_bar_opt[T_train] as given), the DDIM
+ * timesteps tau_i = i * T_train / S (i = 0..S-1; alphas_bar before tau_0 is 1)
+ * and for every step the coefficients of
+ *     x_{tau_{i-1}} = a_i x_{tau_i} + b_i eps + sigma_i z,
+ *     sigma_i = eta sqrt((1-ab_p)/(1-ab_t)) sqrt(1-ab_t/ab_p)
+ * (Song et al., the pages' ref. [7]); uploads a float32 copy.  The schedule
+ * belongs to ctx's device.  Errors: TDM_EINVAL (S < 1, T_train % S != 0,
+ * eta < 0, betas outside (0,1), alphas_bar_opt not decreasing in (0,1)). */
+tdm_status tdm_init_schedule(tdm_ctx *ctx, tdm_schedule **out, int32_t T_train, double beta_start,
+                             double beta_end, const double *alphas_bar_opt, int32_t S, double eta);
+
+void tdm_schedule_destroy(tdm_schedule *sched);
+
+/* Copies the host float64 table, S rows of TDM_SCHED_COLS, into out (host,
+ * n_doubles >= S * TDM_SCHED_COLS). */
+tdm_status tdm_schedule_table(const tdm_schedule *sched, double *out, int64_t n_doubles);
+
+/* Number of DDIM steps S of the schedule (0 for NULL). */
+int32_t tdm_schedule_steps(const tdm_schedule *sched);
+
+/* ---- sampler ----------------------------------------------------------- */
+
+/* Writes the initial state x_T of every map of `tiling` into maps (device,
+ * [C][T][B][64][64]): a symmetric N(0,1) field from the INIT stream (Philox
+ * step word 0).  Entry (i, j), i <= j, is a Box-Muller normal of row quad
+ * (i, j/4); entry (i, j), i > j, repeats entry (j, i). */
+tdm_status tdm_init_noise(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, uint64_t seed,
+                          tdm_stream stream);
+
+/* The stand-in noise prediction of one stream at DDIM step `step`
+ * (0 <= step < S):
+ *     eps_out = (maps - sqrt(ab_t) x0) / sqrt(1 - ab_t) + s * z
+ * with z the symmetric normal field of stream `stream_tag` (TDM_STREAM_EPS_C
+ * or TDM_STREAM_EPS_U) at Philox step word `step`.  maps, eps_out: device
+ * [C][T][B][64][64] (must not overlap); x0: device [C][T][64][64]. */
+tdm_status tdm_eps_standin(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, const float *maps,
+                           const float *x0, float s, int32_t stream_tag, uint64_t seed,
+                           const tdm_tiling *tiling, float *eps_out, tdm_stream stream);
+
+/* One DDIM reverse step `step` (the loop runs step = S-1 .. 0), in place on
+ * maps (device [C][T][B][64][64]):
+ *     eps  = (1 + w) eps_c - w eps_u          (classifier-free guidance, ref. [15])
+ *     maps = a_i maps + b_i eps + sigma_i z   (z: ETA stream, only when eta > 0)
+ * then, when T > 1, sync_every > 0 and (S - step) % sync_every == 0, the
+ * overlap projection of tdm_seam_project.  eps_u may be NULL iff w == 0.
+ * Every map entry is updated (no symmetry is assumed). */
+tdm_status tdm_ddim_step(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, float *maps,
+                         const float *eps_c, const float *eps_u, float w, uint64_t seed,
+                         const tdm_tiling *tiling, tdm_stream stream);
+
+/* The whole reverse run in one launch: for step = S-1 .. 0, the stand-in eps
+ * of both streams (s_c, s_u; the EPS_U stream is not drawn when w == 0), the
+ * guidance combination, the DDIM update and the projection every sync_every
+ * steps.  The state is the folded map -- its upper triangle i <= j, which holds
+ * every bead pair once -- kept in registers for all S steps; on return maps
+ * holds the full symmetric map.  init_noise != 0: x_T is drawn as in
+ * tdm_init_noise; otherwise x_T is read from maps (its upper triangle only).
+ * x0: device [C][T][64][64].  The overlap must be a multiple of 4 (the state
+ * is held in 4-column quads); other overlaps return TDM_EUNSUPPORTED (use
+ * tdm_ddim_step).  Results equal the step-by-step path on symmetric input up
+ * to float32 rounding. */
+tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w,
+                        float s_c, float s_u, uint64_t seed, int32_t init_noise,
+                        const tdm_tiling *tiling, tdm_stream stream);
+
+/* Overlap-consistency projection, in place (ParaChromo §4.3.2, Algorithm 1):
+ * for every chain c, seam k < T-1 and sample b, M = 0.5 * (right block of tile
+ * k + left block of tile k+1), the blocks being rows/cols [64-o, 64) and
+ * [0, o); M is written to both.  Idempotent.  1 <= overlap <= 32. */
+tdm_status tdm_seam_project(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, tdm_stream stream);
+
+/* ---- recovery ------------------------------------------------------------ */
+
+/* Classical MDS of n_maps maps (device [n][64][64]) into coords (device
+ * [n][64][3]) and, if eigvals_opt is not NULL, the top-3 eigenvalues (device
+ * [n][3], descending): D <- (D + D^T)/2, B = -1/2 J (D*D) J, top-3 eigenpairs
+ * (l_k, v_k) of B by subspace iteration with Rayleigh-Ritz, x_k = v_k
+ * sqrt(max(l_k, 0)).  Coordinates are defined up to rotation and reflection.
+ * A map whose eigen-solve does not reach its tolerance within the iteration
+ * cap keeps its last iterate and raises TDM_FLAG_MDS_NOT_CONVERGED. */
+tdm_status tdm_mds_recover(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords,
+                           float *eigvals_opt, tdm_stream stream);
+
+/* maps_out[m][i][j] = || coords[m][i] - coords[m][j] ||_2 (device; zero diagonal). */
+tdm_status tdm_pairwise_dist(tdm_ctx *ctx, const float *coords, int64_t n_maps, float *maps_out,
+                             tdm_stream stream);
+
+/* Seam discrepancy, ParaChromo §5.5 Eq. (6): out[c][k] (device [C][T-1]) =
+ * mean over the o x o overlap of | mean_b right block of tile k - mean_b left
+ * block of tile k+1 |.  Uses context scratch for per-chunk partial sums. */
+tdm_status tdm_seam_discrepancy(tdm_ctx *ctx, const float *maps, const tdm_tiling *tiling, float *out,
+                                tdm_stream stream);
+
+/* The sharded form of Eq. (6): sums (device [C][T-1][o][o]) = sum over this
+ * call's B samples of (right block of tile k - left block of tile k+1).
+ * Sums of several shards add up (e.g. an all-reduce across ranks); then
+ * tdm_seam_discrepancy_finalize divides by tiling->B_total. */
+tdm_status tdm_seam_overlap_sums(tdm_ctx *ctx, const float *maps, const tdm_tiling *tiling, float *sums,
+                                 tdm_stream stream);
+
+tdm_status tdm_seam_discrepancy_finalize(tdm_ctx *ctx, const float *sums, const tdm_tiling *tiling,
+                                         float *out, tdm_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TDM_H */

@@ -1,0 +1,37 @@
+"""Helpers for the GPU parity tests (tolerances, device transfers)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+needs_gpu = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+# Tolerances (normwise per map: max |gpu - oracle| / max |oracle|)
+TOL_MAP = 1e-5        # final and intermediate sampler states
+TOL_NOISE = 2e-6      # a Box-Muller field alone (float32 log/sqrt/sincospi vs float64)
+TOL_RECOVER = 1e-4    # distance maps rebuilt from MDS coordinates; eigenvalues
+TOL_SEAM = 1e-4       # seam discrepancy, relative with a floor
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def host(t):
+    return t.detach().cpu().numpy().astype(np.float64)
+
+
+def normwise(g, o):
+    """Per-map normwise relative error over the last two axes."""
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    num = np.abs(g - o).max(axis=(-1, -2))
+    den = np.maximum(np.abs(o).max(axis=(-1, -2)), 1e-30)
+    return num / den
+
+
+def assert_maps_close(g, o, tol=TOL_MAP, what="maps"):
+    e = normwise(g, o)
+    worst = np.unravel_index(np.argmax(e), e.shape)
+    assert e.max() <= tol, f"{what}: normwise error {e.max():.3e} > {tol:.1e} at {worst}"
+    return e.max()

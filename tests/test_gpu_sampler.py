@@ -1,0 +1,235 @@
+"""GPU parity of the sampler path (init noise, stand-in eps, DDIM step, fused
+run) against the float64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+
+import synth
+from oracle import philox, schedule as osched
+from oracle.ddim import (ddim_run as o_run, eps_standin as o_eps, init_noise as o_init,
+                         sample_ids, stream_noise)
+from tests.gpu_util import (TOL_MAP, TOL_NOISE, assert_maps_close, dev, host, needs_gpu, normwise, torch)
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+@pytest.fixture(scope="module")
+def tdm():
+    import tiled_distance_maps_b200 as m
+    return m
+
+
+def _maps(tiling):
+    return torch.empty(tiling.n_maps * 4096, device="cuda", dtype=torch.float32)
+
+
+def _as5(t, tiling):
+    return host(t).reshape(tiling.C, tiling.T, tiling.B, 64, 64)
+
+
+def test_schedule_table_matches_oracle(tdm):
+    for S, eta in ((50, 0.0), (1000, 1.0), (250, 0.5)):
+        if 1000 % S:
+            continue
+        tab = np.array(tdm.Schedule(S, eta).table())
+        o = osched.Schedule(S=S, eta=eta)
+        np.testing.assert_array_equal(tab[:, 0], o.tau)
+        np.testing.assert_allclose(tab[:, 1], o.ab_t, rtol=1e-14)
+        np.testing.assert_allclose(tab[:, 2], o.ab_p, rtol=1e-14)
+        np.testing.assert_allclose(tab[:, 3], o.sigma, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("base,boff", [(0, 0), (12345, 3)])
+def test_init_noise(tdm, base, boff):
+    t = tdm.Tiling(C=2, T=3, B=4, B_total=9, b_offset=boff, sample_id_base=base)
+    m = _maps(t)
+    tdm.init_noise(m, t, seed=0xDEADBEEF12345)
+    g = _as5(m, t)
+    ids = sample_ids(2, 3, np.arange(boff, boff + 4), 9, base)
+    ref = o_init(0xDEADBEEF12345, ids)
+    assert_maps_close(g, ref, TOL_NOISE, "init noise")
+    np.testing.assert_array_equal(g, np.swapaxes(g, -1, -2))
+
+
+@pytest.mark.parametrize("tag,s", [(1, 0.1), (2, 0.3)])
+def test_eps_standin(tdm, tag, s):
+    t = tdm.Tiling(C=1, T=2, B=3)
+    sch = tdm.Schedule(50)
+    o = osched.Schedule(S=50)
+    x = synth.gaussian_maps(4, 6, symmetric=False).reshape(1, 2, 3, 64, 64) * 3.0
+    x0 = synth.chain_x0(1, 1, 2)
+    out = _maps(t)
+    for step in (49, 20, 0):
+        tdm.eps_standin(sch, step, dev(x), dev(x0), s, tag, 77, t, out)
+        z = stream_noise(77, tag, step, sample_ids(1, 2, np.arange(3), 3))
+        ref = o_eps(x.astype(np.float64), x0[:, :, None].astype(np.float64), o.ab_t[step], s, z)
+        assert_maps_close(_as5(out, t), ref, 1e-5, f"eps step {step}")
+
+
+def _gpu_per_step(tdm, sch, x0, t, w, s_c, s_u, seed, xT=None):
+    """The step-by-step path: init noise, then per step the stand-in eps of
+    each stream and one DDIM step (with the projection when it is due)."""
+    maps = _maps(t)
+    if xT is None:
+        tdm.init_noise(maps, t, seed)
+    else:
+        maps.copy_(dev(xT).reshape(-1))
+    ec, eu = _maps(t), (_maps(t) if w != 0 else None)
+    x0d = dev(x0)
+    states = []
+    for i in reversed(range(sch.S)):
+        tdm.eps_standin(sch, i, maps, x0d, s_c, tdm.STREAM_EPS_C, seed, t, ec)
+        if w != 0:
+            tdm.eps_standin(sch, i, maps, x0d, s_u, tdm.STREAM_EPS_U, seed, t, eu)
+        tdm.ddim_step(sch, i, maps, ec, eu, w, seed, t)
+        states.append(_as5(maps, t))
+    return states
+
+
+def test_per_step_path_small_chain(tdm):
+    # 1 chain x 4 tiles x 8 samples, 50 steps, eta 0, w 0, eps_c noise 0.1,
+    # projection after every step
+    wl = synth.WORKLOADS["chain4_b8_s50"]
+    t = tdm.Tiling(C=1, T=4, B=8, overlap=12, sync_every=1)
+    sch = tdm.Schedule(50)
+    x0 = synth.chain_x0(wl.seed, 1, 4)
+    got = _gpu_per_step(tdm, sch, x0, t, 0.0, 0.1, 0.3, wl.seed)
+    _, traj = o_run(x0, osched.Schedule(S=50), 0.0, 0.1, 0.3, wl.seed, np.arange(8), 8, return_trajectory=True)
+    for n, (g, o) in enumerate(zip(got, traj)):
+        assert_maps_close(g, o, TOL_MAP, f"state after step {n + 1}")
+
+
+def test_per_step_path_cfg_eta_unsymmetric_start(tdm):
+    # w = 1 and eta = 1 exercise both eps streams and the eta stream; a start
+    # that is not symmetric checks that every entry is updated on its own
+    t = tdm.Tiling(C=2, T=3, B=2, overlap=8, sync_every=2)
+    sch = tdm.Schedule(10, eta=1.0)
+    x0 = synth.chain_x0(3, 2, 3, overlap=8)
+    xT = synth.gaussian_maps(9, 12, symmetric=False).reshape(2, 3, 2, 64, 64)
+    got = _gpu_per_step(tdm, sch, x0, t, 1.0, 0.1, 0.3, 5, xT=xT)
+    _, traj = _oracle_unfolded(x0, 10, 1.0, 1.0, 0.1, 0.3, 5, 2, 8, 2, xT)
+    for n, (g, o) in enumerate(zip(got, traj)):
+        assert_maps_close(g, o, TOL_MAP, f"state after step {n + 1}")
+
+
+def _oracle_unfolded(x0, S, eta, w, s_c, s_u, seed, B, overlap, K, xT):
+    """The oracle run on a full (not folded) start state: same steps as
+    oracle.ddim.ddim_run without the fold of x_T."""
+    from oracle.ddim import cfg_combine, ddim_update
+    from oracle.seam import seam_project
+    o = osched.Schedule(S=S, eta=eta)
+    C, T = x0.shape[:2]
+    g = sample_ids(C, T, np.arange(B), B)
+    x = xT.astype(np.float64)
+    x0b = x0[:, :, None].astype(np.float64)
+    traj = []
+    for i in reversed(range(S)):
+        e = o_eps(x, x0b, o.ab_t[i], s_c, stream_noise(seed, philox.TAG_EPS_C, i, g))
+        if w != 0:
+            e = cfg_combine(e, o_eps(x, x0b, o.ab_t[i], s_u, stream_noise(seed, philox.TAG_EPS_U, i, g)), w)
+        z = stream_noise(seed, philox.TAG_ETA, i, g) if eta > 0 else None
+        x = ddim_update(x, e, o.ab_t[i], o.ab_p[i], o.sigma[i], z)
+        if T > 1 and K > 0 and (S - i) % K == 0:
+            x = seam_project(x, overlap)
+        traj.append(x.copy())
+    return x, traj
+
+
+def test_fused_run_small_chain(tdm):
+    wl = synth.WORKLOADS["chain4_b8_s50"]
+    t = tdm.Tiling(C=1, T=4, B=8, overlap=12, sync_every=1)
+    sch = tdm.Schedule(50)
+    x0 = synth.chain_x0(wl.seed, 1, 4)
+    maps = _maps(t)
+    tdm.ddim_run(sch, maps, dev(x0), 0.0, 0.1, 0.3, wl.seed, t)
+    ref = o_run(x0, osched.Schedule(S=50), 0.0, 0.1, 0.3, wl.seed, np.arange(8), 8)
+    g = _as5(maps, t)
+    assert_maps_close(g, ref, TOL_MAP, "fused final maps")
+    np.testing.assert_array_equal(g, np.swapaxes(g, -1, -2))
+    # the final overlap blocks agree exactly after the last projection
+    np.testing.assert_array_equal(g[:, :-1, :, 52:, 52:], g[:, 1:, :, :12, :12])
+
+
+@pytest.mark.parametrize("overlap,K,S,eta,w,T", [(12, 1, 10, 1.0, 0.5, 3), (4, 3, 20, 0.0, 1.0, 4),
+                                                 (32, 2, 5, 1.0, 0.0, 2), (12, 0, 8, 0.0, 1.0, 3),
+                                                 (12, 1, 4, 0.0, 1.0, 1)])
+def test_fused_run_variants_given_start(tdm, overlap, K, S, eta, w, T):
+    C, B = 2, 5
+    t = tdm.Tiling(C=C, T=T, B=B, overlap=overlap, sync_every=K)
+    sch = tdm.Schedule(S, eta=eta)
+    x0 = synth.chain_x0(11, C, T, overlap=overlap)
+    xT = synth.gaussian_maps(13, C * T * B, symmetric=False).reshape(C, T, B, 64, 64)
+    maps = dev(xT).reshape(-1).clone()
+    tdm.ddim_run(sch, maps, dev(x0), w, 0.1, 0.3, 21, t, init_noise=False)
+    ref = o_run(x0, osched.Schedule(S=S, eta=eta), w, 0.1, 0.3, 21, np.arange(B), B, overlap=overlap,
+                sync_every=K, x_T=xT)
+    assert_maps_close(_as5(maps, t), ref, TOL_MAP, "fused final maps")
+
+
+def test_fused_equals_per_step_on_symmetric_start(tdm):
+    t = tdm.Tiling(C=1, T=3, B=4, overlap=12, sync_every=1)
+    sch = tdm.Schedule(25, eta=1.0)
+    x0 = synth.chain_x0(2, 1, 3)
+    fused = _maps(t)
+    tdm.ddim_run(sch, fused, dev(x0), 1.0, 0.1, 0.3, 8, t)
+    per = _gpu_per_step(tdm, sch, x0, t, 1.0, 0.1, 0.3, 8)[-1]
+    assert normwise(_as5(fused, t), per).max() < 2 * TOL_MAP
+
+
+def test_fused_run_is_deterministic_and_shards_reproduce_it(tdm):
+    t = tdm.Tiling(C=1, T=4, B=6, overlap=12, sync_every=1)
+    sch = tdm.Schedule(20)
+    x0 = dev(synth.chain_x0(5, 1, 4))
+    a, b = _maps(t), _maps(t)
+    tdm.ddim_run(sch, a, x0, 1.0, 0.1, 0.3, 3, t)
+    tdm.ddim_run(sch, b, x0, 1.0, 0.1, 0.3, 3, t)
+    torch.testing.assert_close(a, b, rtol=0, atol=0)
+    full = a.view(1, 4, 6, 4096)
+    for b0, nb in ((0, 2), (2, 3), (5, 1)):
+        ts = tdm.Tiling(C=1, T=4, B=nb, overlap=12, sync_every=1, B_total=6, b_offset=b0)
+        part = torch.empty(4 * nb * 4096, device="cuda")
+        tdm.ddim_run(sch, part, x0, 1.0, 0.1, 0.3, 3, ts)
+        torch.testing.assert_close(part.view(1, 4, nb, 4096), full[:, :, b0:b0 + nb], rtol=0, atol=0)
+
+
+def test_chromosome_chain_full_size_sampled(tdm):
+    # 32 tiles x 1000 samples, CFG w=1 (eps_c noise 0.1, eps_u noise 0.3),
+    # 50 steps, projection every step: the launch the benchmark times
+    wl = synth.WORKLOADS["chain32_b1000_cfg"]
+    t = tdm.Tiling(C=1, T=32, B=1000, overlap=12, sync_every=1)
+    sch = tdm.Schedule(50)
+    x0 = synth.chain_x0(wl.seed, 1, 32, sigma=wl.sigma)
+    maps = _maps(t)
+    tdm.ddim_run(sch, maps, dev(x0), wl.w, wl.s_c, wl.s_u, wl.seed, t)
+    g = maps.view(1, 32, 1000, 64, 64)
+    for b in (0, 417, 999):
+        ref = o_run(x0, osched.Schedule(S=50), wl.w, wl.s_c, wl.s_u, wl.seed, [b], 1000)
+        assert_maps_close(host(g[:, :, b:b + 1]), ref, TOL_MAP, f"sample {b}")
+    assert torch.isfinite(g).all()
+
+
+def test_invalid_arguments_are_rejected(tdm):
+    t = tdm.Tiling(C=1, T=2, B=1, overlap=12)
+    sch = tdm.Schedule(10)
+    m = _maps(t)
+    x0 = torch.zeros(2 * 4096, device="cuda")
+    with pytest.raises(tdm.TdmError) as e:
+        tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.3, 0, tdm.Tiling(C=1, T=2, B=1, overlap=10))
+    assert e.value.status == tdm.EUNSUPPORTED
+    with pytest.raises(tdm.TdmError) as e:
+        tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.3, 0, tdm.Tiling(C=1, T=2, B=1, overlap=40))
+    assert e.value.status == tdm.EINVAL
+    with pytest.raises(tdm.TdmError) as e:
+        tdm.ddim_step(sch, 10, m, m, None, 0.0, 0, t)
+    assert e.value.status == tdm.EINVAL
+    with pytest.raises(tdm.TdmError) as e:
+        tdm.ddim_step(sch, 3, m, m, None, 1.0, 0, t)
+    assert e.value.status == tdm.EINVAL
+    with pytest.raises(tdm.TdmError) as e:
+        tdm.Schedule(30)
+    assert e.value.status == tdm.EINVAL
+    with pytest.raises(tdm.TdmError) as e:
+        tdm.ddim_run(sch, m[1:], x0, 0.0, 0.1, 0.3, 0, tdm.Tiling(C=1, T=1, B=1))
+    assert e.value.status == tdm.EINVAL       # misaligned pointer
+    # empty batches are a no-op
+    tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.3, 0, tdm.Tiling(C=0, T=2, B=1))
+    tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.3, 0, tdm.Tiling(C=1, T=2, B=0))

@@ -1,0 +1,473 @@
+// extern "C" entry points of libtdm: argument validation, context, schedule,
+// and dispatch to the kernel launchers.  See include/tdm.h for the contract.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+using tdm::StepCoef;
+using tdm::Tiling;
+
+namespace {
+
+tdm_status fail(tdm_ctx *ctx, tdm_status s, const char *fmt, ...) {
+    if (ctx != nullptr) {
+        char buf[512];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(buf, sizeof(buf), fmt, ap);
+        va_end(ap);
+        ctx->last_error = buf;
+    }
+    return s;
+}
+
+tdm_status cuda_fail(tdm_ctx *ctx, cudaError_t e, const char *where) {
+    return fail(ctx, TDM_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Makes ctx's device current for the scope of an entry point.
+struct DeviceScope {
+    int prev = -1;
+    cudaError_t err = cudaSuccess;
+    explicit DeviceScope(int dev) {
+        err = cudaGetDevice(&prev);
+        if (err == cudaSuccess && prev != dev) err = cudaSetDevice(dev);
+    }
+    ~DeviceScope() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+tdm_status check_tiling(tdm_ctx *ctx, const tdm_tiling *in, Tiling *t) {
+    if (in == nullptr) return fail(ctx, TDM_EINVAL, "tiling is NULL");
+    if (in->C < 0 || in->T < 1 || in->B < 0)
+        return fail(ctx, TDM_EINVAL, "tiling: need C >= 0, T >= 1, B >= 0 (got %d, %d, %d)", in->C, in->T, in->B);
+    if (in->reserved != 0) return fail(ctx, TDM_EINVAL, "tiling: reserved field must be 0");
+    if (in->T > 1 && (in->overlap < 1 || in->overlap > 32))
+        return fail(ctx, TDM_EINVAL, "tiling: overlap must be in [1, 32] (got %d)", in->overlap);
+    if (in->T == 1 && (in->overlap < 0 || in->overlap > 32))
+        return fail(ctx, TDM_EINVAL, "tiling: overlap must be in [0, 32] (got %d)", in->overlap);
+    if (in->T > 0xFFFF) return fail(ctx, TDM_EUNSUPPORTED, "tiling: at most 65535 tiles per chain");
+    if (in->sync_every < 0) return fail(ctx, TDM_EINVAL, "tiling: sync_every must be >= 0");
+    const int64_t B_total = in->B_total == 0 ? in->B : in->B_total;
+    if (in->b_offset < 0 || in->sample_id_base < 0 || B_total < in->b_offset + in->B)
+        return fail(ctx, TDM_EINVAL, "tiling: need 0 <= b_offset, b_offset + B <= B_total, sample_id_base >= 0");
+    // every noise id must fit the 56 bits of the Philox counter
+    const long double max_id = (long double)in->sample_id_base +
+                               ((long double)in->C * in->T) * (long double)B_total;
+    if (max_id > (long double)(1ULL << 56))
+        return fail(ctx, TDM_EUNSUPPORTED, "tiling: noise ids exceed 2^56");
+    t->C = in->C;
+    t->T = in->T;
+    t->B = in->B;
+    t->overlap = in->overlap;
+    t->sync_every = in->sync_every;
+    t->B_total = B_total;
+    t->b_offset = in->b_offset;
+    t->sample_id_base = in->sample_id_base;
+    return TDM_OK;
+}
+
+tdm_status check_maps(tdm_ctx *ctx, const void *p, const char *name) {
+    if (p == nullptr) return fail(ctx, TDM_EINVAL, "%s is NULL", name);
+    if (!aligned16(p)) return fail(ctx, TDM_EINVAL, "%s is not 16-byte aligned", name);
+    return TDM_OK;
+}
+
+tdm_status check_sched(tdm_ctx *ctx, const tdm_schedule *s) {
+    if (s == nullptr || s->d_coef == nullptr) return fail(ctx, TDM_EINVAL, "schedule is NULL");
+    if (s->device != ctx->device) return fail(ctx, TDM_EINVAL, "schedule belongs to another device");
+    return TDM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tdm_status_str(tdm_status s) {
+    switch (s) {
+        case TDM_OK: return "ok";
+        case TDM_EINVAL: return "invalid argument";
+        case TDM_ECUDA: return "CUDA error";
+        case TDM_ETIMEOUT: return "timed out";
+        case TDM_ENONFINITE: return "non-finite value";
+        case TDM_EUNSUPPORTED: return "unsupported";
+        case TDM_ENOMEM: return "out of device memory";
+        case TDM_ENOTCONVERGED: return "eigen-solve did not converge";
+        default: return "unknown status";
+    }
+}
+
+const char *tdm_ctx_last_error(const tdm_ctx *ctx) { return ctx == nullptr ? "" : ctx->last_error.c_str(); }
+
+tdm_status tdm_ctx_create(tdm_ctx **out, int32_t device) {
+    if (out == nullptr) return TDM_EINVAL;
+    *out = nullptr;
+    int count = 0;
+    if (cudaGetDeviceCount(&count) != cudaSuccess || device < 0 || device >= count) return TDM_EINVAL;
+    tdm_ctx *ctx = new (std::nothrow) tdm_ctx();
+    if (ctx == nullptr) return TDM_ENOMEM;
+    ctx->device = device;
+    DeviceScope ds(device);
+    if (ds.err != cudaSuccess) {
+        delete ctx;
+        return TDM_ECUDA;
+    }
+    // scratch: per-chunk partial sums of the seam discrepancy (<= 1184 seam
+    // chunks of up to 32 x 32 entries)
+    ctx->scratch_floats = (size_t)1184 * 1024;
+    if (cudaMalloc(&ctx->d_flags, sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_scratch, ctx->scratch_floats * sizeof(float)) != cudaSuccess ||
+        cudaMemset(ctx->d_flags, 0, sizeof(uint32_t)) != cudaSuccess) {
+        cudaFree(ctx->d_flags);
+        cudaFree(ctx->d_scratch);
+        delete ctx;
+        cudaGetLastError();
+        return TDM_ENOMEM;
+    }
+    *out = ctx;
+    return TDM_OK;
+}
+
+void tdm_ctx_destroy(tdm_ctx *ctx) {
+    if (ctx == nullptr) return;
+    {
+        DeviceScope ds(ctx->device);
+        for (auto &kv : ctx->plans) cudaFree(kv.second);
+        cudaFree(ctx->d_flags);
+        cudaFree(ctx->d_scratch);
+    }
+    delete ctx;
+}
+
+tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    DeviceScope ds(ctx->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "stream synchronize");
+    uint32_t flags = 0;
+    e = cudaMemcpy(&flags, ctx->d_flags, sizeof(flags), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(ctx->d_flags, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "status word");
+    if (flags_out != nullptr) *flags_out = flags;
+    if (flags & TDM_FLAG_MDS_NOT_CONVERGED)
+        return fail(ctx, TDM_ENOTCONVERGED, "an MDS eigen-solve reached its iteration cap");
+    return TDM_OK;
+}
+
+// ---- schedule -----------------------------------------------------------------------
+
+tdm_status tdm_init_schedule(tdm_ctx *ctx, tdm_schedule **out, int32_t T_train, double beta_start,
+                             double beta_end, const double *alphas_bar_opt, int32_t S, double eta) {
+    if (ctx == nullptr || out == nullptr) return fail(ctx, TDM_EINVAL, "ctx or out is NULL");
+    *out = nullptr;
+    if (T_train < 1 || S < 1 || S > T_train || T_train % S != 0)
+        return fail(ctx, TDM_EINVAL, "schedule: need 1 <= S, S divides T_train (got T=%d, S=%d)", T_train, S);
+    if (!(eta >= 0.0) || !std::isfinite(eta)) return fail(ctx, TDM_EINVAL, "schedule: eta must be >= 0");
+    std::vector<double> ab((size_t)T_train);
+    if (alphas_bar_opt == nullptr) {
+        if (!(beta_start > 0.0 && beta_start < 1.0 && beta_end > 0.0 && beta_end < 1.0))
+            return fail(ctx, TDM_EINVAL, "schedule: betas must lie in (0, 1)");
+        double acc = 1.0;
+        for (int t = 0; t < T_train; ++t) {
+            const double b = T_train > 1 ? beta_start + (beta_end - beta_start) * (double)t / (double)(T_train - 1)
+                                         : beta_start;
+            acc *= (1.0 - b);
+            ab[(size_t)t] = acc;
+        }
+    } else {
+        double prev = 1.0;
+        for (int t = 0; t < T_train; ++t) {
+            const double v = alphas_bar_opt[t];
+            if (!(v > 0.0 && v < prev)) return fail(ctx, TDM_EINVAL, "schedule: alphas_bar must decrease in (0, 1)");
+            ab[(size_t)t] = prev = v;
+        }
+    }
+    tdm_schedule *s = new (std::nothrow) tdm_schedule();
+    if (s == nullptr) return fail(ctx, TDM_ENOMEM, "schedule: host allocation");
+    s->device = ctx->device;
+    s->T_train = T_train;
+    s->S = S;
+    s->eta = eta;
+    s->table.assign((size_t)S * TDM_SCHED_COLS, 0.0);
+    std::vector<StepCoef> coef((size_t)S);
+    const int stride = T_train / S;
+    for (int i = 0; i < S; ++i) {
+        const int tau = i * stride;
+        const double ab_t = ab[(size_t)tau];
+        const double ab_p = i > 0 ? ab[(size_t)(tau - stride)] : 1.0;
+        const double sigma = eta * std::sqrt((1.0 - ab_p) / (1.0 - ab_t)) * std::sqrt(1.0 - ab_t / ab_p);
+        const double a = std::sqrt(ab_p) / std::sqrt(ab_t);
+        const double dir = 1.0 - ab_p - sigma * sigma;
+        const double b = std::sqrt(dir > 0.0 ? dir : 0.0) - std::sqrt(ab_p) * std::sqrt(1.0 - ab_t) / std::sqrt(ab_t);
+        const double sa = std::sqrt(ab_t), isa1 = 1.0 / std::sqrt(1.0 - ab_t);
+        double *row = &s->table[(size_t)i * TDM_SCHED_COLS];
+        row[0] = tau;
+        row[1] = ab_t;
+        row[2] = ab_p;
+        row[3] = sigma;
+        row[4] = a;
+        row[5] = b;
+        row[6] = sa;
+        row[7] = isa1;
+        StepCoef &c = coef[(size_t)i];
+        c.ka = (float)(a + b * isa1);
+        c.kx0 = (float)(-b * isa1 * sa);
+        c.kb = (float)b;
+        c.ks = (float)sigma;
+        c.a = (float)a;
+        c.sa = (float)sa;
+        c.isa1 = (float)isa1;
+        c.pad = 0.0f;
+    }
+    DeviceScope ds(ctx->device);
+    cudaError_t e = cudaMalloc(&s->d_coef, sizeof(StepCoef) * (size_t)S);
+    if (e == cudaSuccess) e = cudaMemcpy(s->d_coef, coef.data(), sizeof(StepCoef) * (size_t)S, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(s->d_coef);
+        delete s;
+        return cuda_fail(ctx, e, "schedule upload");
+    }
+    *out = s;
+    return TDM_OK;
+}
+
+void tdm_schedule_destroy(tdm_schedule *s) {
+    if (s == nullptr) return;
+    {
+        DeviceScope ds(s->device);
+        cudaFree(s->d_coef);
+    }
+    delete s;
+}
+
+tdm_status tdm_schedule_table(const tdm_schedule *s, double *out, int64_t n) {
+    if (s == nullptr || out == nullptr || n < (int64_t)s->table.size()) return TDM_EINVAL;
+    std::memcpy(out, s->table.data(), s->table.size() * sizeof(double));
+    return TDM_OK;
+}
+
+int32_t tdm_schedule_steps(const tdm_schedule *s) { return s == nullptr ? 0 : s->S; }
+
+// ---- sampler ------------------------------------------------------------------------
+
+tdm_status tdm_init_noise(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, uint64_t seed, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    Tiling t;
+    tdm_status s = check_tiling(ctx, tiling, &t);
+    if (s != TDM_OK) return s;
+    if (t.n_maps() == 0) return TDM_OK;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_init_noise(maps, t, seed, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "init_noise launch");
+}
+
+tdm_status tdm_eps_standin(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, const float *maps,
+                           const float *x0, float s_noise, int32_t stream_tag, uint64_t seed,
+                           const tdm_tiling *tiling, float *eps_out, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    tdm_status s = check_sched(ctx, sched);
+    if (s != TDM_OK) return s;
+    Tiling t;
+    if ((s = check_tiling(ctx, tiling, &t)) != TDM_OK) return s;
+    if (step < 0 || step >= sched->S) return fail(ctx, TDM_EINVAL, "step %d outside [0, %d)", step, sched->S);
+    if (stream_tag != TDM_STREAM_EPS_C && stream_tag != TDM_STREAM_EPS_U)
+        return fail(ctx, TDM_EINVAL, "stream_tag must be TDM_STREAM_EPS_C or TDM_STREAM_EPS_U");
+    if (!std::isfinite(s_noise)) return fail(ctx, TDM_EINVAL, "noise scale is not finite");
+    if (t.n_maps() == 0) return TDM_OK;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, x0, "x0")) != TDM_OK ||
+        (s = check_maps(ctx, eps_out, "eps_out")) != TDM_OK)
+        return s;
+    if (eps_out == maps) return fail(ctx, TDM_EINVAL, "eps_out must not alias maps");
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_eps_standin(sched->d_coef, step, maps, x0, s_noise, stream_tag, seed, t, eps_out,
+                                            static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "eps_standin launch");
+}
+
+tdm_status tdm_seam_project(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    Tiling t;
+    tdm_status s = check_tiling(ctx, tiling, &t);
+    if (s != TDM_OK) return s;
+    if (t.n_maps() == 0 || t.T < 2) return TDM_OK;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_seam_project(maps, t, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "seam_project launch");
+}
+
+tdm_status tdm_ddim_step(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, float *maps, const float *eps_c,
+                         const float *eps_u, float w, uint64_t seed, const tdm_tiling *tiling, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    tdm_status s = check_sched(ctx, sched);
+    if (s != TDM_OK) return s;
+    Tiling t;
+    if ((s = check_tiling(ctx, tiling, &t)) != TDM_OK) return s;
+    if (step < 0 || step >= sched->S) return fail(ctx, TDM_EINVAL, "step %d outside [0, %d)", step, sched->S);
+    if (!std::isfinite(w)) return fail(ctx, TDM_EINVAL, "w is not finite");
+    if (w != 0.0f && eps_u == nullptr) return fail(ctx, TDM_EINVAL, "eps_u is NULL but w != 0");
+    if (t.n_maps() == 0) return TDM_OK;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, eps_c, "eps_c")) != TDM_OK)
+        return s;
+    if (w != 0.0f && (s = check_maps(ctx, eps_u, "eps_u")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tdm::launch_ddim_step(sched->d_coef, step, maps, eps_c, w != 0.0f ? eps_u : nullptr, w,
+                                          sched->eta > 0.0, seed, t, st);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "ddim_step launch");
+    if (t.T > 1 && t.sync_every > 0 && (sched->S - step) % t.sync_every == 0) {
+        e = tdm::launch_seam_project(maps, t, st);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "seam projection launch");
+    }
+    return TDM_OK;
+}
+
+tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w, float s_c,
+                        float s_u, uint64_t seed, int32_t init_noise, const tdm_tiling *tiling, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    tdm_status s = check_sched(ctx, sched);
+    if (s != TDM_OK) return s;
+    Tiling t;
+    if ((s = check_tiling(ctx, tiling, &t)) != TDM_OK) return s;
+    if (!std::isfinite(w) || !std::isfinite(s_c) || !std::isfinite(s_u))
+        return fail(ctx, TDM_EINVAL, "w, s_c, s_u must be finite");
+    if (t.T > 1 && t.overlap % 4 != 0)
+        return fail(ctx, TDM_EUNSUPPORTED, "ddim_run: overlap must be a multiple of 4 (got %d)", t.overlap);
+    if (t.n_maps() == 0) return TDM_OK;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, x0, "x0")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    const int ov = t.T > 1 ? t.overlap : 0;
+    uint32_t *plan = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(ctx->mu);
+        auto it = ctx->plans.find({t.T, ov});
+        if (it != ctx->plans.end()) {
+            plan = it->second;
+        } else {
+            std::vector<uint32_t> h = tdm::build_run_plan(t.T, ov);
+            if (h.size() != (size_t)tdm::kUpperQuads * t.T)
+                return fail(ctx, TDM_EUNSUPPORTED, "ddim_run: lane plan has wrong size");
+            cudaError_t e = cudaMalloc(&plan, h.size() * sizeof(uint32_t));
+            if (e == cudaSuccess) e = cudaMemcpy(plan, h.data(), h.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
+            if (e != cudaSuccess) {
+                cudaFree(plan);
+                return cuda_fail(ctx, e, "lane plan upload");
+            }
+            ctx->plans[{t.T, ov}] = plan;
+        }
+    }
+    cudaError_t e = tdm::launch_ddim_run(sched->d_coef, sched->S, maps, x0, w, s_c, s_u, sched->eta > 0.0, seed,
+                                         init_noise != 0, t, plan, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "ddim_run launch");
+}
+
+// ---- recovery -----------------------------------------------------------------------
+
+tdm_status tdm_mds_recover(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, float *eigvals_opt,
+                           tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (n_maps < 0) return fail(ctx, TDM_EINVAL, "n_maps < 0");
+    if (n_maps == 0) return TDM_OK;
+    tdm_status s;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, coords, "coords")) != TDM_OK) return s;
+    if (eigvals_opt != nullptr && (reinterpret_cast<uintptr_t>(eigvals_opt) & 3u))
+        return fail(ctx, TDM_EINVAL, "eigvals is not 4-byte aligned");
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_mds(maps, n_maps, coords, eigvals_opt, ctx->d_flags, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "mds launch");
+}
+
+tdm_status tdm_pairwise_dist(tdm_ctx *ctx, const float *coords, int64_t n_maps, float *maps_out, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (n_maps < 0) return fail(ctx, TDM_EINVAL, "n_maps < 0");
+    if (n_maps == 0) return TDM_OK;
+    tdm_status s;
+    if ((s = check_maps(ctx, coords, "coords")) != TDM_OK || (s = check_maps(ctx, maps_out, "maps_out")) != TDM_OK)
+        return s;
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_pdist(coords, n_maps, maps_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "pairwise_dist launch");
+}
+
+tdm_status tdm_seam_overlap_sums(tdm_ctx *ctx, const float *maps, const tdm_tiling *tiling, float *sums,
+                                 tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    Tiling t;
+    tdm_status s = check_tiling(ctx, tiling, &t);
+    if (s != TDM_OK) return s;
+    if (t.T < 2) return fail(ctx, TDM_EINVAL, "seam sums need T >= 2");
+    if ((int64_t)t.C * (t.T - 1) == 0) return TDM_OK;
+    if ((s = check_maps(ctx, sums, "sums")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (t.B == 0) {
+        cudaError_t e = cudaMemsetAsync(sums, 0, sizeof(float) * (size_t)t.C * (t.T - 1) * t.overlap * t.overlap, st);
+        return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "seam sums clear");
+    }
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK) return s;
+    const int64_t n_seams = (int64_t)t.C * (t.T - 1);
+    const int oo = t.overlap * t.overlap;
+    int chunks = tdm::seam_chunks(n_seams, t.B);
+    cudaError_t e;
+    if (chunks > 1 && (size_t)n_seams * chunks * oo <= ctx->scratch_floats) {
+        e = tdm::launch_seam_sums(maps, t, ctx->d_scratch, chunks, st);
+        if (e == cudaSuccess) e = tdm::launch_seam_reduce(ctx->d_scratch, t, chunks, sums, st);
+    } else {
+        e = tdm::launch_seam_sums(maps, t, sums, 1, st);
+    }
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "seam sums launch");
+}
+
+tdm_status tdm_seam_discrepancy_finalize(tdm_ctx *ctx, const float *sums, const tdm_tiling *tiling, float *out,
+                                         tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    Tiling t;
+    tdm_status s = check_tiling(ctx, tiling, &t);
+    if (s != TDM_OK) return s;
+    if (t.T < 2) return fail(ctx, TDM_EINVAL, "seam discrepancy needs T >= 2");
+    if (t.B_total < 1) return fail(ctx, TDM_EINVAL, "seam discrepancy needs B_total >= 1");
+    if ((int64_t)t.C * (t.T - 1) == 0) return TDM_OK;
+    if ((s = check_maps(ctx, sums, "sums")) != TDM_OK || (s = check_maps(ctx, out, "out")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_seam_finalize(sums, t, 1, 1.0 / (double)t.B_total, out,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "seam finalize launch");
+}
+
+tdm_status tdm_seam_discrepancy(tdm_ctx *ctx, const float *maps, const tdm_tiling *tiling, float *out,
+                                tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    Tiling t;
+    tdm_status s = check_tiling(ctx, tiling, &t);
+    if (s != TDM_OK) return s;
+    if (t.T < 2) return fail(ctx, TDM_EINVAL, "seam discrepancy needs T >= 2");
+    if (t.B < 1) return fail(ctx, TDM_EINVAL, "seam discrepancy needs B >= 1");
+    if ((int64_t)t.C * (t.T - 1) == 0) return TDM_OK;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, out, "out")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n_seams = (int64_t)t.C * (t.T - 1);
+    const int oo = t.overlap * t.overlap;
+    const int chunks = tdm::seam_chunks(n_seams, t.B);
+    const double inv_b = 1.0 / (double)t.B;
+    cudaError_t e;
+    if (chunks > 1 && (size_t)n_seams * chunks * oo <= ctx->scratch_floats) {
+        e = tdm::launch_seam_sums(maps, t, ctx->d_scratch, chunks, st);
+        if (e == cudaSuccess) e = tdm::launch_seam_finalize(ctx->d_scratch, t, chunks, inv_b, out, st);
+    } else {
+        e = tdm::launch_seam_finalize(maps, t, 0, inv_b, out, st);
+    }
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "seam discrepancy launch");
+}
+
+}  // extern "C"

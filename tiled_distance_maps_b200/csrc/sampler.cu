@@ -1,0 +1,394 @@
+// Sampler kernels: initial noise, stand-in eps, one DDIM step, and the fused
+// whole-trajectory run.
+//
+// ParaChromo (mdpi.com/2079-9292/15/13/2750): the reverse chain runs DDIM at a
+// reduced step count (§4.1, §5.1.1) with classifier-free guidance (§3.1, ref.
+// [15]); tiled regions are coupled only through the overlap projection of
+// §4.3.2.  The stand-in eps is the ideal denoiser toward x0 plus Philox noise.
+#include "common.cuh"
+
+namespace tdm {
+namespace {
+
+__device__ const UpperQuadTable kUpperQuadTable = make_upper_quads();
+
+constexpr int kMapThreads = 256;   // CTA size of the one-map-per-iteration kernels
+constexpr int kZLd = kN + 1;       // row stride of the symmetric noise tile in smem
+
+
+// Fills zs[64][65] with the symmetric normal field of map noise id g.
+__device__ __forceinline__ void fill_symmetric_noise(float *zs, uint64_t g, int tag, uint32_t step_word,
+                                                     uint32_t k0, uint32_t k1) {
+    for (int u = threadIdx.x; u < kUpperQuads; u += blockDim.x) {
+        const int rq = kUpperQuadTable.v[u];
+        const int r = rq >> 4, q = rq & 15;
+        const float4 z = quad_normals(r, q, step_word, g, tag, k0, k1);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int j = 4 * q + t;
+            if (j >= r) {
+                zs[r * kZLd + j] = comp(z, t);
+                zs[j * kZLd + r] = comp(z, t);
+            }
+        }
+    }
+}
+
+// ---- initial state ---------------------------------------------------------
+
+__global__ void __launch_bounds__(256) init_noise_kernel(float *__restrict__ maps, int64_t n_maps, int T,
+                                                         int B, int64_t B_total, int64_t b_off,
+                                                         int64_t base, uint32_t k0, uint32_t k1) {
+    const int64_t total = n_maps * kUpperQuads;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = idx / kUpperQuads;
+        const int u = (int)(idx - m * kUpperQuads);
+        const int rq = kUpperQuadTable.v[u];
+        const int r = rq >> 4, q = rq & 15;
+        const int64_t tile = m / B;
+        const int b = (int)(m - tile * B);
+        const int c = (int)(tile / T), k = (int)(tile - (int64_t)c * T);
+        const uint64_t g = noise_id(base, c, T, k, B_total, b_off, b);
+        const float4 z = quad_normals(r, q, 0u, g, TDM_STREAM_INIT, k0, k1);
+        float *mp = maps + m * kMapFloats;
+        if (4 * q > r) {
+            st4(mp + r * kN + 4 * q, z);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mp[(4 * q + t) * kN + r] = comp(z, t);
+        } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int j = 4 * q + t;
+                if (j >= r) mp[r * kN + j] = comp(z, t);
+                if (j > r) mp[j * kN + r] = comp(z, t);
+            }
+        }
+    }
+}
+
+// ---- stand-in eps of one stream ---------------------------------------------
+
+__global__ void __launch_bounds__(kMapThreads) eps_standin_kernel(
+    const StepCoef *__restrict__ coef, int step, const float *__restrict__ maps, const float *__restrict__ x0,
+    float s, int tag, uint32_t k0, uint32_t k1, Tiling t, float *__restrict__ eps) {
+    __shared__ float zs[kN * kZLd];
+    const StepCoef cf = coef[step];
+    const int64_t n = t.n_maps();
+    for (int64_t m = blockIdx.x; m < n; m += gridDim.x) {
+        const int64_t tile = m / t.B;
+        const int b = (int)(m - tile * t.B);
+        const int c = (int)(tile / t.T), k = (int)(tile - (int64_t)c * t.T);
+        const uint64_t g = noise_id(t.sample_id_base, c, t.T, k, t.B_total, t.b_offset, b);
+        fill_symmetric_noise(zs, g, tag, (uint32_t)step, k0, k1);
+        __syncthreads();
+        const float *xm = maps + m * kMapFloats;
+        const float *x0m = x0 + tile * kMapFloats;
+        float *em = eps + m * kMapFloats;
+#pragma unroll 4
+        for (int p = threadIdx.x; p < kMapFloats / 4; p += kMapThreads) {
+            const int r = p >> 4, q = p & 15;
+            const float4 x = ld4(xm + 4 * p);
+            const float4 xr = ldg4(x0m + 4 * p);
+            const float *z = zs + r * kZLd + 4 * q;
+            float4 e;
+            e.x = fmaf(s, z[0], (x.x - cf.sa * xr.x) * cf.isa1);
+            e.y = fmaf(s, z[1], (x.y - cf.sa * xr.y) * cf.isa1);
+            e.z = fmaf(s, z[2], (x.z - cf.sa * xr.z) * cf.isa1);
+            e.w = fmaf(s, z[3], (x.w - cf.sa * xr.w) * cf.isa1);
+            st4(em + 4 * p, e);
+        }
+        __syncthreads();
+    }
+}
+
+// ---- one DDIM step ------------------------------------------------------------
+
+template <bool HAS_U, bool HAS_ETA>
+__global__ void __launch_bounds__(kMapThreads) ddim_step_kernel(
+    const StepCoef *__restrict__ coef, int step, float *__restrict__ maps, const float *__restrict__ eps_c,
+    const float *__restrict__ eps_u, float w, uint32_t k0, uint32_t k1, Tiling t) {
+    __shared__ float zs[HAS_ETA ? kN * kZLd : 1];
+    const StepCoef cf = coef[step];
+    const float wc = 1.0f + w;
+    const int64_t n = t.n_maps();
+    for (int64_t m = blockIdx.x; m < n; m += gridDim.x) {
+        if (HAS_ETA) {
+            const int64_t tile = m / t.B;
+            const int b = (int)(m - tile * t.B);
+            const int c = (int)(tile / t.T), k = (int)(tile - (int64_t)c * t.T);
+            const uint64_t g = noise_id(t.sample_id_base, c, t.T, k, t.B_total, t.b_offset, b);
+            fill_symmetric_noise(zs, g, TDM_STREAM_ETA, (uint32_t)step, k0, k1);
+            __syncthreads();
+        }
+        float *xm = maps + m * kMapFloats;
+        const float *ec = eps_c + m * kMapFloats;
+        const float *eu = HAS_U ? eps_u + m * kMapFloats : nullptr;
+#pragma unroll 4
+        for (int p = threadIdx.x; p < kMapFloats / 4; p += kMapThreads) {
+            float4 x = ld4(xm + 4 * p);
+            float4 e = ldg4(ec + 4 * p);
+            if (HAS_U) {
+                const float4 v = ldg4(eu + 4 * p);
+                e.x = wc * e.x - w * v.x;
+                e.y = wc * e.y - w * v.y;
+                e.z = wc * e.z - w * v.z;
+                e.w = wc * e.w - w * v.w;
+            }
+            x.x = fmaf(cf.a, x.x, cf.kb * e.x);
+            x.y = fmaf(cf.a, x.y, cf.kb * e.y);
+            x.z = fmaf(cf.a, x.z, cf.kb * e.z);
+            x.w = fmaf(cf.a, x.w, cf.kb * e.w);
+            if (HAS_ETA) {
+                const float *z = zs + (p >> 4) * kZLd + 4 * (p & 15);
+                x.x = fmaf(cf.ks, z[0], x.x);
+                x.y = fmaf(cf.ks, z[1], x.y);
+                x.z = fmaf(cf.ks, z[2], x.z);
+                x.w = fmaf(cf.ks, z[3], x.w);
+            }
+            st4(xm + 4 * p, x);
+        }
+        if (HAS_ETA) __syncthreads();
+    }
+}
+
+// ---- the fused whole-trajectory run -------------------------------------------
+//
+// One lane owns one row quad (r, 4q..4q+3) of the folded (upper-triangle)
+// state of one map and keeps it in registers for all S steps.  With the
+// stand-in denoiser every update is elementwise, so the only coupling between
+// lanes is the overlap projection, which pairs entry (s+i, s+j) of tile k with
+// entry (i, j) of tile k+1 of the same sample.  The lane plan puts both quads
+// of such a pair in lanes l and l^16 of one warp, so the projection is one
+// register exchange; no CTA ever waits on another.
+
+struct RunArgs {
+    const StepCoef *coef;
+    float *maps;
+    const float *x0;
+    const uint32_t *plan;      // [17 T][32] lane descriptors
+    int64_t total_warps;       // C * B * 17 T
+    int64_t B_total, b_off, base;
+    int S, T, B, sync_every, warps_per_chain;
+    float cc, cu;              // (1 + w) s_c and w s_u
+    uint32_t k0, k1;
+};
+
+template <bool HAS_U, bool HAS_ETA, bool INIT>
+__global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
+    extern __shared__ float4 sco[];        // [S] (ka, kx0, kc, ku) then [S] ks
+    float *sks = reinterpret_cast<float *>(sco + a.S);
+    for (int i = threadIdx.x; i < a.S; i += blockDim.x) {
+        const StepCoef c = a.coef[i];
+        sco[i] = make_float4(c.ka, c.kx0, c.kb * a.cc, -(c.kb * a.cu));
+        if (HAS_ETA) sks[i] = c.ks;
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (gw >= a.total_warps) return;
+    const int64_t cs = gw / a.warps_per_chain;               // chain-sample c * B + b
+    const int wi = (int)(gw - cs * a.warps_per_chain);
+    const uint32_t d = __ldg(a.plan + wi * 32 + lane);
+    const int q = d & 15, r = (d >> 4) & 63, k = (d >> 10) & 0xFFFF;
+    const bool paired = (d >> 31) != 0;
+    const int c = (int)(cs / a.B), b = (int)(cs - (int64_t)c * a.B);
+    const int64_t tile = (int64_t)c * a.T + k;
+    float *mp = a.maps + (tile * a.B + b) * kMapFloats;
+    const uint64_t g = (uint64_t)(a.base + tile * a.B_total + a.b_off + b);
+    const float4 xr = ldg4(a.x0 + tile * kMapFloats + r * kN + 4 * q);
+
+    float4 x = INIT ? quad_normals(r, q, 0u, g, TDM_STREAM_INIT, a.k0, a.k1) : ld4(mp + r * kN + 4 * q);
+    const bool tiled = a.T > 1 && a.sync_every > 0;
+
+    for (int i = a.S - 1; i >= 0; --i) {
+        const float4 cf = sco[i];
+        const float4 zc = quad_normals(r, q, (uint32_t)i, g, TDM_STREAM_EPS_C, a.k0, a.k1);
+        float4 acc;
+        acc.x = fmaf(cf.z, zc.x, cf.y * xr.x);
+        acc.y = fmaf(cf.z, zc.y, cf.y * xr.y);
+        acc.z = fmaf(cf.z, zc.z, cf.y * xr.z);
+        acc.w = fmaf(cf.z, zc.w, cf.y * xr.w);
+        if (HAS_U) {
+            const float4 zu = quad_normals(r, q, (uint32_t)i, g, TDM_STREAM_EPS_U, a.k0, a.k1);
+            acc.x = fmaf(cf.w, zu.x, acc.x);
+            acc.y = fmaf(cf.w, zu.y, acc.y);
+            acc.z = fmaf(cf.w, zu.z, acc.z);
+            acc.w = fmaf(cf.w, zu.w, acc.w);
+        }
+        if (HAS_ETA) {
+            const float ks = sks[i];
+            const float4 ze = quad_normals(r, q, (uint32_t)i, g, TDM_STREAM_ETA, a.k0, a.k1);
+            acc.x = fmaf(ks, ze.x, acc.x);
+            acc.y = fmaf(ks, ze.y, acc.y);
+            acc.z = fmaf(ks, ze.z, acc.z);
+            acc.w = fmaf(ks, ze.w, acc.w);
+        }
+        x.x = fmaf(cf.x, x.x, acc.x);
+        x.y = fmaf(cf.x, x.y, acc.y);
+        x.z = fmaf(cf.x, x.z, acc.z);
+        x.w = fmaf(cf.x, x.w, acc.w);
+        if (tiled && (a.S - i) % a.sync_every == 0) {
+            float4 o;
+            o.x = __shfl_xor_sync(0xffffffffu, x.x, 16);
+            o.y = __shfl_xor_sync(0xffffffffu, x.y, 16);
+            o.z = __shfl_xor_sync(0xffffffffu, x.z, 16);
+            o.w = __shfl_xor_sync(0xffffffffu, x.w, 16);
+            if (paired) {
+                x.x = 0.5f * (x.x + o.x);
+                x.y = 0.5f * (x.y + o.y);
+                x.z = 0.5f * (x.z + o.z);
+                x.w = 0.5f * (x.w + o.w);
+            }
+        }
+    }
+
+    // unfold: the quad's upper entries go to (r, j) and their mirrors to (j, r)
+    if (4 * q > r) {
+        st4(mp + r * kN + 4 * q, x);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mp[(4 * q + t) * kN + r] = comp(x, t);
+    } else {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int j = 4 * q + t;
+            if (j >= r) mp[r * kN + j] = comp(x, t);
+            if (j > r) mp[j * kN + r] = comp(x, t);
+        }
+    }
+}
+
+int grid_for(int64_t work_items, int per_sm) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = (int64_t)sms * per_sm;
+    return (int)(work_items < cap ? (work_items > 0 ? work_items : 1) : cap);
+}
+
+}  // namespace
+
+// ---- host side -------------------------------------------------------------------
+
+std::vector<uint32_t> build_run_plan(int T, int overlap) {
+    const int s = kN - overlap, sq = s / 4, oq = overlap / 4;
+    auto desc = [](int k, int r, int q, bool paired) {
+        return (uint32_t)q | ((uint32_t)r << 4) | ((uint32_t)k << 10) | (paired ? 0x80000000u : 0u);
+    };
+    std::vector<std::pair<uint32_t, uint32_t>> pairs;
+    std::vector<uint32_t> singles;
+    for (int k = 0; k < T; ++k)
+        for (int r = 0; r < kN; ++r)
+            for (int q = 0; q < kQuadsPerRow; ++q) {
+                if (4 * q + 3 < r) continue;                       // not in the folded state
+                const bool right = k < T - 1 && r >= s && q >= sq;
+                const bool left = k > 0 && r < overlap && q < oq;
+                if (right)
+                    pairs.emplace_back(desc(k, r, q, true), desc(k + 1, r - s, q - sq, true));
+                else if (!left)
+                    singles.push_back(desc(k, r, q, false));
+            }
+    std::vector<uint32_t> plan;
+    plan.reserve((size_t)kUpperQuads * T);
+    size_t si = 0;
+    for (size_t p0 = 0; p0 < pairs.size(); p0 += 16) {
+        uint32_t wl[32];
+        for (int l = 0; l < 16; ++l) {
+            if (p0 + l < pairs.size()) {
+                wl[l] = pairs[p0 + l].first;
+                wl[l + 16] = pairs[p0 + l].second;
+            } else {
+                wl[l] = singles[si++];
+                wl[l + 16] = singles[si++];
+            }
+        }
+        plan.insert(plan.end(), wl, wl + 32);
+    }
+    plan.insert(plan.end(), singles.begin() + si, singles.end());
+    return plan;
+}
+
+cudaError_t launch_init_noise(float *maps, const Tiling &t, uint64_t seed, cudaStream_t st) {
+    const int64_t items = t.n_maps() * kUpperQuads;
+    const int grid = grid_for((items + 255) / 256, 16);
+    init_noise_kernel<<<grid, 256, 0, st>>>(maps, t.n_maps(), t.T, t.B, t.B_total, t.b_offset,
+                                            t.sample_id_base, (uint32_t)seed, (uint32_t)(seed >> 32));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_eps_standin(const StepCoef *coef, int step, const float *maps, const float *x0, float s,
+                               int tag, uint64_t seed, const Tiling &t, float *eps, cudaStream_t st) {
+    const int grid = grid_for(t.n_maps(), 8);
+    eps_standin_kernel<<<grid, kMapThreads, 0, st>>>(coef, step, maps, x0, s, tag, (uint32_t)seed,
+                                                     (uint32_t)(seed >> 32), t, eps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ddim_step(const StepCoef *coef, int step, float *maps, const float *eps_c,
+                             const float *eps_u, float w, bool has_eta, uint64_t seed, const Tiling &t,
+                             cudaStream_t st) {
+    const int grid = grid_for(t.n_maps(), 8);
+    const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    const bool has_u = eps_u != nullptr && w != 0.0f;
+    if (has_u && has_eta)
+        ddim_step_kernel<true, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, k0, k1, t);
+    else if (has_u)
+        ddim_step_kernel<true, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, k0, k1, t);
+    else if (has_eta)
+        ddim_step_kernel<false, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, k0, k1, t);
+    else
+        ddim_step_kernel<false, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, k0, k1, t);
+    return cudaGetLastError();
+}
+
+template <bool U, bool E, bool I>
+static cudaError_t run_variant(const RunArgs &a, int grid, size_t smem, cudaStream_t st) {
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(ddim_run_kernel<U, E, I>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    ddim_run_kernel<U, E, I><<<grid, 256, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ddim_run(const StepCoef *coef, int S, float *maps, const float *x0, float w, float s_c,
+                            float s_u, bool has_eta, uint64_t seed, bool init_noise, const Tiling &t,
+                            const uint32_t *plan, cudaStream_t st) {
+    RunArgs a;
+    a.coef = coef;
+    a.maps = maps;
+    a.x0 = x0;
+    a.plan = plan;
+    a.warps_per_chain = 17 * t.T;
+    a.total_warps = (int64_t)t.C * t.B * a.warps_per_chain;
+    a.B_total = t.B_total;
+    a.b_off = t.b_offset;
+    a.base = t.sample_id_base;
+    a.S = S;
+    a.T = t.T;
+    a.B = t.B;
+    a.sync_every = t.sync_every;
+    a.cc = (1.0f + w) * s_c;
+    a.cu = w * s_u;
+    a.k0 = (uint32_t)seed;
+    a.k1 = (uint32_t)(seed >> 32);
+    const int64_t grid64 = (a.total_warps + 7) / 8;
+    if (grid64 > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+    const int grid = (int)grid64;
+    const size_t smem = (size_t)S * (sizeof(float4) + (has_eta ? sizeof(float) : 0));
+    const bool has_u = w != 0.0f;
+    if (has_u) {
+        if (has_eta) return init_noise ? run_variant<true, true, true>(a, grid, smem, st)
+                                       : run_variant<true, true, false>(a, grid, smem, st);
+        return init_noise ? run_variant<true, false, true>(a, grid, smem, st)
+                          : run_variant<true, false, false>(a, grid, smem, st);
+    }
+    if (has_eta) return init_noise ? run_variant<false, true, true>(a, grid, smem, st)
+                                   : run_variant<false, true, false>(a, grid, smem, st);
+    return init_noise ? run_variant<false, false, true>(a, grid, smem, st)
+                      : run_variant<false, false, false>(a, grid, smem, st);
+}
+
+}  // namespace tdm
