@@ -15,9 +15,10 @@ reading of that, written out in the design notes:
 
 where ``g`` is the map's global sample id, ``tag`` the noise stream and
 ``(row, quad)`` a row-aligned group of four columns ``4*quad .. 4*quad+3``.
-Each output word pair (a, b) gives two normals by Box-Muller on 24-bit
-uniforms u1 = (a>>8 + 1) / 2^24 in (0, 1] and u2 = (b>>8) / 2^24 in [0, 1):
-r = sqrt(-2 ln u1), z0 = r cos(2 pi u2), z1 = r sin(2 pi u2).
+Each output word pair (a, b) gives two normals by Box-Muller on 23-bit
+uniforms u1 = 1 - (a>>9) / 2^23 in (0, 1] and u2 = (b>>9) / 2^23 in [0, 1):
+r = sqrt(-2 ln u1), z0 = r cos(2 pi u2), z1 = r sin(2 pi u2).  (23 bits: both
+uniforms are then exact float32 numbers built from a float's mantissa.)
 """
 from __future__ import annotations
 
@@ -63,8 +64,8 @@ def box_muller(a, b):
     """Two standard normals from two 32-bit words (float64)."""
     a = np.asarray(a, dtype=np.uint64)
     b = np.asarray(b, dtype=np.uint64)
-    u1 = ((a >> np.uint64(8)) + np.uint64(1)).astype(np.float64) / 16777216.0
-    u2 = (b >> np.uint64(8)).astype(np.float64) / 16777216.0
+    u1 = 1.0 - (a >> np.uint64(9)).astype(np.float64) / 8388608.0
+    u2 = (b >> np.uint64(9)).astype(np.float64) / 8388608.0
     r = np.sqrt(-2.0 * np.log(u1))
     return r * np.cos(2.0 * np.pi * u2), r * np.sin(2.0 * np.pi * u2)
 

@@ -68,21 +68,24 @@ def test_philox_matches_triton_library():
 
 
 def test_box_muller_special_values():
-    # a = 0xFFFFFFFF -> u1 = 1 -> r = 0
-    z0, z1 = philox.box_muller(0xFFFFFFFF, 12345 << 8)
+    # a>>9 = 0 -> u1 = 1 -> r = 0
+    z0, z1 = philox.box_muller(0x000001FF, 12345 << 9)
     assert z0 == 0.0 and z1 == 0.0
-    # a = 0 -> u1 = 2^-24 -> r = sqrt(2 * 24 ln 2); b = 0 -> angle 0
-    r = np.sqrt(48.0 * np.log(2.0))
-    z0, z1 = philox.box_muller(0, 0)
-    assert abs(z0 - r) < 1e-15 and z1 == 0.0
-    # b>>8 = 2^22 -> u2 = 1/4 -> angle pi/2
-    z0, z1 = philox.box_muller(0, 1 << 30)
+    # a>>9 = 2^23 - 1 -> u1 = 2^-23 -> r = sqrt(2 * 23 ln 2); b = 0 -> angle 0
+    r = np.sqrt(46.0 * np.log(2.0))
+    z0, z1 = philox.box_muller(0xFFFFFFFF, 0)
+    assert abs(z0 - r) < 1e-14 and z1 == 0.0
+    # b>>9 = 2^21 -> u2 = 1/4 -> angle pi/2
+    z0, z1 = philox.box_muller(0xFFFFFFFF, 1 << 30)
     assert abs(z0) < 1e-14 and abs(z1 - r) < 1e-14
-    # b>>8 = 2^23 -> u2 = 1/2 -> angle pi
-    z0, z1 = philox.box_muller(0, 1 << 31)
+    # b>>9 = 2^22 -> u2 = 1/2 -> angle pi
+    z0, z1 = philox.box_muller(0xFFFFFFFF, 1 << 31)
     assert abs(z0 + r) < 1e-14 and abs(z1) < 1e-14
-    # the low 8 bits of either word are ignored
-    assert philox.box_muller(0x12345678, 0x9ABCDEF0) == philox.box_muller(0x123456FF, 0x9ABCDE00)
+    # a>>9 = 2^22 -> u1 = 1/2 -> r = sqrt(2 ln 2)
+    z0, _ = philox.box_muller(1 << 31, 0)
+    assert abs(z0 - np.sqrt(2.0 * np.log(2.0))) < 1e-15
+    # the low 9 bits of either word are ignored
+    assert philox.box_muller(0x12345678, 0x9ABCDEF0) == philox.box_muller(0x123457FF, 0x9ABCDE00)
 
 
 def test_normals_are_standard():
@@ -95,8 +98,8 @@ def test_normals_are_standard():
     assert abs(v.mean()) < 5.0 / np.sqrt(v.size)
     assert abs(v.var() - 1.0) < 6.0 * np.sqrt(2.0 / v.size)
     assert stats.kstest(v[:200000], "norm").pvalue > 1e-4
-    # the tail is cut at r = sqrt(48 ln 2) ~ 5.77
-    assert np.abs(v).max() <= np.sqrt(48.0 * np.log(2.0)) + 1e-12
+    # the tail is cut at r = sqrt(46 ln 2) ~ 5.65
+    assert np.abs(v).max() <= np.sqrt(46.0 * np.log(2.0)) + 1e-12
 
 
 def test_streams_steps_and_samples_are_independent():
