@@ -36,13 +36,18 @@ METRIC = "map-denoise-steps/sec (64-bead fp32 maps) on 1 B200; % FP32/HBM roofli
 UNIT = "map-steps/s"
 
 # Algorithmic operations of one quad-step of the fused run (one 4-entry row
-# quad of the folded state advanced one DDIM step), counted per lane:
-#   Philox4x32-10 call: 10 rounds x (2 mul.wide + 4 xor + 2 key adds) + 3 counter ops = 83
-#   Box-Muller pair: 2 shifts, 1 add, 2 int->float, 2 scales, log, mul, sqrt,
-#                    mul, sincospi, 2 muls = 15
-#   one noise stream per quad: 83 + 2 x 15 = 113
-#   update: one FMA per entry per term (x_t, x0, each noise stream)
-OPS_PHILOX = 83
+# quad of the folded state advanced one DDIM step), counted per lane as the
+# fewest hardware instructions that the formulation needs (one per 32x32->64
+# multiply, 3-input xor, float add/multiply/FMA, shift, or, and MUFU
+# transcendental):
+#   Philox4x32-10 call: 10 rounds x (2 wide multiplies + 2 three-input xors) = 40
+#   Box-Muller pair: 2 words x (shift + or + subtract) + (1 - e) + log2 + scale
+#                    + sqrt + angle scale + sin + cos + 2 products = 15
+#   one noise stream per quad: 40 + 2 x 15 = 70
+#   update: one FMA per entry per term (x_t, x0 and each noise stream)
+# Guards that only serve accuracy (the small-e series, the clamp at 0) and
+# loop or address work are not counted, so the fraction is a lower bound.
+OPS_PHILOX = 40
 OPS_BOX_MULLER_PAIR = 15
 QUADS_PER_MAP = 544
 

@@ -180,6 +180,22 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
  * [0, o); M is written to both.  Idempotent.  1 <= overlap <= 32. */
 tdm_status tdm_seam_project(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, tdm_stream stream);
 
+/* ---- noise primitives ----------------------------------------------------
+ * The two stages of every noise stream, on caller data, so that a caller can
+ * reproduce any noise value and check the transform's error exhaustively. */
+
+/* out[i] = Philox4x32-10(ctr[i], key = (seed mod 2^32, seed div 2^32)) (Salmon
+ * et al., SC'11); ctr, out: device uint32 [n][4], 16-byte aligned. */
+tdm_status tdm_philox4x32(tdm_ctx *ctx, const uint32_t *ctr, int64_t n, uint64_t seed, uint32_t *out,
+                          tdm_stream stream);
+
+/* The uniform-to-normal transform of every stream: for word pair (a, b) =
+ * words[2i], words[2i+1], u1 = 1 - (a>>9) 2^-23, u2 = (b>>9) 2^-23,
+ * z[2i] = sqrt(-2 ln u1) cos(2 pi u2), z[2i+1] = sqrt(-2 ln u1) sin(2 pi u2),
+ * evaluated with float32 hardware approximations.  words: device uint32
+ * [n_pairs][2]; z: device float32 [n_pairs][2]; both 8-byte aligned. */
+tdm_status tdm_box_muller(tdm_ctx *ctx, const uint32_t *words, int64_t n_pairs, float *z, tdm_stream stream);
+
 /* ---- recovery ------------------------------------------------------------ */
 
 /* Classical MDS of n_maps maps (device [n][64][64]) into coords (device

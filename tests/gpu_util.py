@@ -8,7 +8,9 @@ needs_gpu = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CU
 
 # Tolerances (normwise per map: max |gpu - oracle| / max |oracle|)
 TOL_MAP = 1e-5        # final and intermediate sampler states
-TOL_NOISE = 2e-6      # a Box-Muller field alone (float32 log/sqrt/sincospi vs float64)
+# absolute bound on one float32 normal against float64: |dr| + r_max |d angle|
+# with the exhaustively measured bounds of tests/test_gpu_noise.py
+Z_ABS_ERR = 4e-6 + 5.65 * 1.5e-6
 TOL_RECOVER = 1e-4    # distance maps rebuilt from MDS coordinates; eigenvalues
 TOL_SEAM = 1e-4       # seam discrepancy, relative with a floor
 

@@ -21,8 +21,8 @@ def declared():
 @pytest.fixture(scope="module")
 def lib():
     if not os.path.exists(LIB):
-        from tiled_distance_maps_b200 import build
-        build.build(quiet=True)
+        import __graft_entry__
+        __graft_entry__._build_module().build(quiet=True)
     return ctypes.CDLL(LIB)
 
 

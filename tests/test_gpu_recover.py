@@ -89,10 +89,24 @@ def test_pairwise_dist_matches_oracle(tdm):
 
 
 def test_recovery_of_sampler_output(tdm):
-    # MDS and reconstruction of the final maps of the small tiled chain
+    # the whole pipeline on the small tiled chain: GPU sampler -> GPU MDS ->
+    # GPU reconstruction against oracle sampler -> oracle MDS -> oracle
+    # reconstruction, each side from the same synthetic x0
+    from oracle import schedule as osched
+    from oracle.ddim import ddim_run as o_run
     wl = synth.WORKLOADS["chain4_b8_s50"]
     t = tdm.Tiling(C=1, T=4, B=8)
     sch = tdm.Schedule(50)
-    maps = torch.empty(t.n_maps * 4096, device="cuda")
-    tdm.ddim_run(sch, maps, dev(synth.chain_x0(wl.seed, 1, 4)), 0.0, 0.1, 0.3, wl.seed, t)
-    _check(tdm, host(maps).reshape(-1, 64, 64).astype(np.float32), "sampler output")
+    x0 = synth.chain_x0(wl.seed, 1, 4)
+    n = t.n_maps
+    maps = torch.empty(n * 4096, device="cuda")
+    coords = torch.empty(n * 192, device="cuda")
+    rec = torch.empty(n * 4096, device="cuda")
+    tdm.ddim_run(sch, maps, dev(x0), 0.0, 0.1, 0.3, wl.seed, t)
+    tdm.mds_recover(maps, n, coords)
+    tdm.pairwise_dist(coords, n, rec)
+    assert tdm.ctx_sync() == 0
+    ref = o_run(x0, osched.Schedule(S=50), 0.0, 0.1, 0.3, wl.seed, np.arange(8), 8).reshape(-1, 64, 64)
+    Xo, _ = omds.classical_mds(ref)
+    e = normwise(host(rec).reshape(-1, 64, 64), omds.pairwise_distances(Xo))
+    assert e.max() <= TOL_RECOVER, e.max()

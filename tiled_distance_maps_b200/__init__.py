@@ -7,7 +7,7 @@ is no CPU path.  Tensors must be CUDA float32, contiguous, 16-byte aligned.
 PyTorch is used only for device memory and streams.
 
 Importing the package loads ``libtdm.so`` and raises ImportError when it is
-missing (build it with ``python -m tiled_distance_maps_b200.build``).
+missing or stale (build it with ``python tiled_distance_maps_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libtdm.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libtdm.so not found at {LIB_PATH}; build it with "
-                      "`python -m tiled_distance_maps_b200.build`")
+                      "`python tiled_distance_maps_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, EINVAL, ECUDA, ETIMEOUT, ENONFINITE, EUNSUPPORTED, ENOMEM, ENOTCONVERGED = range(8)
@@ -59,9 +59,15 @@ _SIGS = {
     "tdm_seam_discrepancy": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp]),
     "tdm_seam_overlap_sums": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp]),
     "tdm_seam_discrepancy_finalize": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp]),
+    "tdm_philox4x32": (_i32, [_vp, _vp, _i64, _u64, _vp, _vp]),
+    "tdm_box_muller": (_i32, [_vp, _vp, _i64, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
-    _fn = getattr(_lib, _name)
+    try:
+        _fn = getattr(_lib, _name)
+    except AttributeError as _e:
+        raise ImportError(f"{LIB_PATH} does not export {_name}; rebuild it with "
+                          "`python tiled_distance_maps_b200/build.py`") from _e
     _fn.restype = _res
     _fn.argtypes = _args
 
@@ -317,6 +323,37 @@ def seam_discrepancy_finalize(sums, tiling: Tiling, out, ctx: Context | None = N
     ctx.check(_lib.tdm_seam_discrepancy_finalize(ctx.handle, _ptr(sums, "sums", ctx), ctypes.byref(ct),
                                                  _ptr(out, "out", ctx), _stream(ctx)))
     return out
+
+
+def _uptr(t, name, ctx, dtype):
+    import torch
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    return _vp(t.data_ptr())
+
+
+def philox4x32(ctr, seed: int, out, ctx: Context | None = None):
+    """out[i] = Philox4x32-10(ctr[i], seed); ctr, out: CUDA uint32 [n, 4]."""
+    import torch
+    ctx = ctx or context(ctr.device.index)
+    n = ctr.numel() // 4
+    if out.numel() < 4 * n:
+        raise ValueError("out too small")
+    ctx.check(_lib.tdm_philox4x32(ctx.handle, _uptr(ctr, "ctr", ctx, torch.uint32), n, int(seed),
+                                  _uptr(out, "out", ctx, torch.uint32), _stream(ctx)))
+    return out
+
+
+def box_muller(words, z, ctx: Context | None = None):
+    """z[2i], z[2i+1] from words[2i], words[2i+1]; words CUDA uint32, z float32."""
+    import torch
+    ctx = ctx or context(words.device.index)
+    n = words.numel() // 2
+    if z.numel() < 2 * n:
+        raise ValueError("z too small")
+    ctx.check(_lib.tdm_box_muller(ctx.handle, _uptr(words, "words", ctx, torch.uint32), n,
+                                  _uptr(z, "z", ctx, torch.float32), _stream(ctx)))
+    return z
 
 
 def ctx_sync(ctx: Context | None = None) -> int:

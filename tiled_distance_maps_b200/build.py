@@ -1,6 +1,8 @@
 """Builds libtdm.so in-tree with nvcc for sm_100a.
 
-    python -m tiled_distance_maps_b200.build [--force] [--ptxas-verbose]
+    python tiled_distance_maps_b200/build.py [--force] [--ptxas-verbose]
+
+(run as a script: importing the package would load the library being built)
 
 Objects go to ``_build/`` at the repository root; the shared library is written
 next to this file so that it travels with the source tree.

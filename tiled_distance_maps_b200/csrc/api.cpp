@@ -371,6 +371,32 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "ddim_run launch");
 }
 
+// ---- noise primitives ---------------------------------------------------------------
+
+tdm_status tdm_philox4x32(tdm_ctx *ctx, const uint32_t *ctr, int64_t n, uint64_t seed, uint32_t *out,
+                          tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (n < 0) return fail(ctx, TDM_EINVAL, "n < 0");
+    if (n == 0) return TDM_OK;
+    tdm_status s;
+    if ((s = check_maps(ctx, ctr, "ctr")) != TDM_OK || (s = check_maps(ctx, out, "out")) != TDM_OK) return s;
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_philox(ctr, n, seed, out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "philox launch");
+}
+
+tdm_status tdm_box_muller(tdm_ctx *ctx, const uint32_t *words, int64_t n_pairs, float *z, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (n_pairs < 0) return fail(ctx, TDM_EINVAL, "n_pairs < 0");
+    if (n_pairs == 0) return TDM_OK;
+    if (words == nullptr || z == nullptr || (reinterpret_cast<uintptr_t>(words) & 7u) ||
+        (reinterpret_cast<uintptr_t>(z) & 7u))
+        return fail(ctx, TDM_EINVAL, "words and z must be non-NULL and 8-byte aligned");
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_box_muller(words, n_pairs, z, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "box_muller launch");
+}
+
 // ---- recovery -----------------------------------------------------------------------
 
 tdm_status tdm_mds_recover(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, float *eigvals_opt,

@@ -18,11 +18,11 @@ constexpr int kZLd = kN + 1;       // row stride of the symmetric noise tile in 
 
 // Fills zs[64][65] with the symmetric normal field of map noise id g.
 __device__ __forceinline__ void fill_symmetric_noise(float *zs, uint64_t g, int tag, uint32_t step_word,
-                                                     uint32_t k0, uint32_t k1) {
+                                                     const PhiloxKeys &K) {
     for (int u = threadIdx.x; u < kUpperQuads; u += blockDim.x) {
         const int rq = kUpperQuadTable.v[u];
         const int r = rq >> 4, q = rq & 15;
-        const float4 z = quad_normals(r, q, step_word, g, tag, k0, k1);
+        const float4 z = quad_normals(r, q, step_word, g, tag, K);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const int j = 4 * q + t;
@@ -38,7 +38,7 @@ __device__ __forceinline__ void fill_symmetric_noise(float *zs, uint64_t g, int 
 
 __global__ void __launch_bounds__(256) init_noise_kernel(float *__restrict__ maps, int64_t n_maps, int T,
                                                          int B, int64_t B_total, int64_t b_off,
-                                                         int64_t base, uint32_t k0, uint32_t k1) {
+                                                         int64_t base, const PhiloxKeys K) {
     const int64_t total = n_maps * kUpperQuads;
     for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) init_noise_kernel(float *__restrict__ map
         const int b = (int)(m - tile * B);
         const int c = (int)(tile / T), k = (int)(tile - (int64_t)c * T);
         const uint64_t g = noise_id(base, c, T, k, B_total, b_off, b);
-        const float4 z = quad_normals(r, q, 0u, g, TDM_STREAM_INIT, k0, k1);
+        const float4 z = quad_normals(r, q, 0u, g, TDM_STREAM_INIT, K);
         float *mp = maps + m * kMapFloats;
         if (4 * q > r) {
             st4(mp + r * kN + 4 * q, z);
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256) init_noise_kernel(float *__restrict__ map
 
 __global__ void __launch_bounds__(kMapThreads) eps_standin_kernel(
     const StepCoef *__restrict__ coef, int step, const float *__restrict__ maps, const float *__restrict__ x0,
-    float s, int tag, uint32_t k0, uint32_t k1, Tiling t, float *__restrict__ eps) {
+    float s, int tag, const PhiloxKeys K, Tiling t, float *__restrict__ eps) {
     __shared__ float zs[kN * kZLd];
     const StepCoef cf = coef[step];
     const int64_t n = t.n_maps();
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(kMapThreads) eps_standin_kernel(
         const int b = (int)(m - tile * t.B);
         const int c = (int)(tile / t.T), k = (int)(tile - (int64_t)c * t.T);
         const uint64_t g = noise_id(t.sample_id_base, c, t.T, k, t.B_total, t.b_offset, b);
-        fill_symmetric_noise(zs, g, tag, (uint32_t)step, k0, k1);
+        fill_symmetric_noise(zs, g, tag, (uint32_t)step, K);
         __syncthreads();
         const float *xm = maps + m * kMapFloats;
         const float *x0m = x0 + tile * kMapFloats;
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kMapThreads) eps_standin_kernel(
 template <bool HAS_U, bool HAS_ETA>
 __global__ void __launch_bounds__(kMapThreads) ddim_step_kernel(
     const StepCoef *__restrict__ coef, int step, float *__restrict__ maps, const float *__restrict__ eps_c,
-    const float *__restrict__ eps_u, float w, uint32_t k0, uint32_t k1, Tiling t) {
+    const float *__restrict__ eps_u, float w, const PhiloxKeys K, Tiling t) {
     __shared__ float zs[HAS_ETA ? kN * kZLd : 1];
     const StepCoef cf = coef[step];
     const float wc = 1.0f + w;
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kMapThreads) ddim_step_kernel(
             const int b = (int)(m - tile * t.B);
             const int c = (int)(tile / t.T), k = (int)(tile - (int64_t)c * t.T);
             const uint64_t g = noise_id(t.sample_id_base, c, t.T, k, t.B_total, t.b_offset, b);
-            fill_symmetric_noise(zs, g, TDM_STREAM_ETA, (uint32_t)step, k0, k1);
+            fill_symmetric_noise(zs, g, TDM_STREAM_ETA, (uint32_t)step, K);
             __syncthreads();
         }
         float *xm = maps + m * kMapFloats;
@@ -171,8 +171,43 @@ struct RunArgs {
     int64_t B_total, b_off, base;
     int S, T, B, sync_every, warps_per_chain;
     float cc, cu;              // (1 + w) s_c and w s_u
-    uint32_t k0, k1;
+    PhiloxKeys K;
 };
+
+// Round 1 of Philox for a lane whose counter words 0 (position) and 2 (noise
+// id, low half) never change: its products are computed once, and the round-1
+// output for step word i and stream tag t is (A ^ i, L1, B ^ t << 24, L0).
+struct LaneCounter {
+    uint32_t A, L1, B, L0;
+};
+
+__device__ __forceinline__ LaneCounter lane_counter(int r, int q, uint64_t g, const PhiloxKeys &K) {
+    const uint64_t p0 = (uint64_t)Philox::M0 * (((uint32_t)r << 4) | (uint32_t)q);
+    const uint64_t p1 = (uint64_t)Philox::M1 * (uint32_t)g;
+    LaneCounter L;
+    L.A = (uint32_t)(p1 >> 32) ^ K.k0[0];
+    L.L1 = (uint32_t)p1;
+    L.B = (uint32_t)(p0 >> 32) ^ ((uint32_t)(g >> 32) & 0xFFFFFFu) ^ K.k1[0];
+    L.L0 = (uint32_t)p0;
+    return L;
+}
+
+// The normals of NS streams (tags TAGS...) of one step for one lane: the
+// streams share counter words 0 and 1, so round 2's first product is shared.
+template <int NS>
+__device__ __forceinline__ void lane_normals(const LaneCounter &L, uint32_t step_word, const int (&tags)[NS],
+                                             const PhiloxKeys &K, float4 (&z)[NS]) {
+    const uint64_t p0 = (uint64_t)Philox::M0 * (L.A ^ step_word);
+    const uint32_t w2 = (uint32_t)(p0 >> 32) ^ L.L0 ^ K.k1[1];
+    const uint32_t w3 = (uint32_t)p0;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+        const uint64_t p1 = (uint64_t)Philox::M1 * (L.B ^ ((uint32_t)tags[s] << 24));
+        uint4 c = make_uint4((uint32_t)(p1 >> 32) ^ L.L1 ^ K.k0[1], (uint32_t)p1, w2, w3);
+        c = philox_rounds<2>(c, K);
+        z[s] = words_to_normals(c);
+    }
+}
 
 template <bool HAS_U, bool HAS_ETA, bool INIT>
 __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
@@ -198,28 +233,47 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     float *mp = a.maps + (tile * a.B + b) * kMapFloats;
     const uint64_t g = (uint64_t)(a.base + tile * a.B_total + a.b_off + b);
     const float4 xr = ldg4(a.x0 + tile * kMapFloats + r * kN + 4 * q);
+    const LaneCounter L = lane_counter(r, q, g, a.K);
 
-    float4 x = INIT ? quad_normals(r, q, 0u, g, TDM_STREAM_INIT, a.k0, a.k1) : ld4(mp + r * kN + 4 * q);
-    const bool tiled = a.T > 1 && a.sync_every > 0;
+    float4 x;
+    if (INIT) {
+        constexpr int kInit[1] = {TDM_STREAM_INIT};
+        float4 z0[1];
+        lane_normals<1>(L, 0u, kInit, a.K, z0);
+        x = z0[0];
+    } else {
+        x = ld4(mp + r * kN + 4 * q);
+    }
+    // only warps that hold seam pairs (lane 0 is paired in every such warp of
+    // the plan) take part in the projection
+    const bool warp_pairs = __shfl_sync(0xffffffffu, paired ? 1 : 0, 0) != 0;
+    const bool sync_warp = a.T > 1 && a.sync_every > 0 && warp_pairs;
+    int until_sync = a.sync_every;
+
+    constexpr int NS = 1 + (HAS_U ? 1 : 0) + (HAS_ETA ? 1 : 0);
+    constexpr int kTags[3] = {TDM_STREAM_EPS_C, HAS_U ? TDM_STREAM_EPS_U : TDM_STREAM_ETA, TDM_STREAM_ETA};
+    int tags[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) tags[s] = kTags[s];
 
     for (int i = a.S - 1; i >= 0; --i) {
         const float4 cf = sco[i];
-        const float4 zc = quad_normals(r, q, (uint32_t)i, g, TDM_STREAM_EPS_C, a.k0, a.k1);
+        float4 z[NS];
+        lane_normals<NS>(L, (uint32_t)i, tags, a.K, z);
         float4 acc;
-        acc.x = fmaf(cf.z, zc.x, cf.y * xr.x);
-        acc.y = fmaf(cf.z, zc.y, cf.y * xr.y);
-        acc.z = fmaf(cf.z, zc.z, cf.y * xr.z);
-        acc.w = fmaf(cf.z, zc.w, cf.y * xr.w);
+        acc.x = fmaf(cf.z, z[0].x, cf.y * xr.x);
+        acc.y = fmaf(cf.z, z[0].y, cf.y * xr.y);
+        acc.z = fmaf(cf.z, z[0].z, cf.y * xr.z);
+        acc.w = fmaf(cf.z, z[0].w, cf.y * xr.w);
         if (HAS_U) {
-            const float4 zu = quad_normals(r, q, (uint32_t)i, g, TDM_STREAM_EPS_U, a.k0, a.k1);
-            acc.x = fmaf(cf.w, zu.x, acc.x);
-            acc.y = fmaf(cf.w, zu.y, acc.y);
-            acc.z = fmaf(cf.w, zu.z, acc.z);
-            acc.w = fmaf(cf.w, zu.w, acc.w);
+            acc.x = fmaf(cf.w, z[1].x, acc.x);
+            acc.y = fmaf(cf.w, z[1].y, acc.y);
+            acc.z = fmaf(cf.w, z[1].z, acc.z);
+            acc.w = fmaf(cf.w, z[1].w, acc.w);
         }
         if (HAS_ETA) {
             const float ks = sks[i];
-            const float4 ze = quad_normals(r, q, (uint32_t)i, g, TDM_STREAM_ETA, a.k0, a.k1);
+            const float4 ze = z[NS - 1];
             acc.x = fmaf(ks, ze.x, acc.x);
             acc.y = fmaf(ks, ze.y, acc.y);
             acc.z = fmaf(ks, ze.z, acc.z);
@@ -229,7 +283,8 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
         x.y = fmaf(cf.x, x.y, acc.y);
         x.z = fmaf(cf.x, x.z, acc.z);
         x.w = fmaf(cf.x, x.w, acc.w);
-        if (tiled && (a.S - i) % a.sync_every == 0) {
+        if (sync_warp && --until_sync == 0) {
+            until_sync = a.sync_every;
             float4 o;
             o.x = __shfl_xor_sync(0xffffffffu, x.x, 16);
             o.y = __shfl_xor_sync(0xffffffffu, x.y, 16);
@@ -256,6 +311,22 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
             if (j >= r) mp[r * kN + j] = comp(x, t);
             if (j > r) mp[j * kN + r] = comp(x, t);
         }
+    }
+}
+
+// ---- the noise primitives on caller words (for exhaustive checks) -------------
+
+__global__ void __launch_bounds__(256) philox_kernel(const uint4 *__restrict__ ctr, int64_t n, const PhiloxKeys K,
+                                                     uint4 *__restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        out[i] = philox4x32_10(ctr[i], K);
+}
+
+__global__ void __launch_bounds__(256) box_muller_kernel(const uint2 *__restrict__ words, int64_t n,
+                                                         float2 *__restrict__ z) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint2 w = words[i];
+        z[i] = box_muller(w.x, w.y);
     }
 }
 
@@ -313,15 +384,14 @@ cudaError_t launch_init_noise(float *maps, const Tiling &t, uint64_t seed, cudaS
     const int64_t items = t.n_maps() * kUpperQuads;
     const int grid = grid_for((items + 255) / 256, 16);
     init_noise_kernel<<<grid, 256, 0, st>>>(maps, t.n_maps(), t.T, t.B, t.B_total, t.b_offset,
-                                            t.sample_id_base, (uint32_t)seed, (uint32_t)(seed >> 32));
+                                            t.sample_id_base, philox_keys(seed));
     return cudaGetLastError();
 }
 
 cudaError_t launch_eps_standin(const StepCoef *coef, int step, const float *maps, const float *x0, float s,
                                int tag, uint64_t seed, const Tiling &t, float *eps, cudaStream_t st) {
     const int grid = grid_for(t.n_maps(), 8);
-    eps_standin_kernel<<<grid, kMapThreads, 0, st>>>(coef, step, maps, x0, s, tag, (uint32_t)seed,
-                                                     (uint32_t)(seed >> 32), t, eps);
+    eps_standin_kernel<<<grid, kMapThreads, 0, st>>>(coef, step, maps, x0, s, tag, philox_keys(seed), t, eps);
     return cudaGetLastError();
 }
 
@@ -329,16 +399,16 @@ cudaError_t launch_ddim_step(const StepCoef *coef, int step, float *maps, const 
                              const float *eps_u, float w, bool has_eta, uint64_t seed, const Tiling &t,
                              cudaStream_t st) {
     const int grid = grid_for(t.n_maps(), 8);
-    const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    const PhiloxKeys K = philox_keys(seed);
     const bool has_u = eps_u != nullptr && w != 0.0f;
     if (has_u && has_eta)
-        ddim_step_kernel<true, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, k0, k1, t);
+        ddim_step_kernel<true, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, K, t);
     else if (has_u)
-        ddim_step_kernel<true, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, k0, k1, t);
+        ddim_step_kernel<true, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, K, t);
     else if (has_eta)
-        ddim_step_kernel<false, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, k0, k1, t);
+        ddim_step_kernel<false, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, K, t);
     else
-        ddim_step_kernel<false, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, k0, k1, t);
+        ddim_step_kernel<false, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, K, t);
     return cudaGetLastError();
 }
 
@@ -372,8 +442,7 @@ cudaError_t launch_ddim_run(const StepCoef *coef, int S, float *maps, const floa
     a.sync_every = t.sync_every;
     a.cc = (1.0f + w) * s_c;
     a.cu = w * s_u;
-    a.k0 = (uint32_t)seed;
-    a.k1 = (uint32_t)(seed >> 32);
+    a.K = philox_keys(seed);
     const int64_t grid64 = (a.total_warps + 7) / 8;
     if (grid64 > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
     const int grid = (int)grid64;
@@ -389,6 +458,26 @@ cudaError_t launch_ddim_run(const StepCoef *coef, int S, float *maps, const floa
                                    : run_variant<false, true, false>(a, grid, smem, st);
     return init_noise ? run_variant<false, false, true>(a, grid, smem, st)
                       : run_variant<false, false, false>(a, grid, smem, st);
+}
+
+}  // namespace tdm
+
+namespace tdm {
+
+cudaError_t launch_philox(const uint32_t *ctr, int64_t n, uint64_t seed, uint32_t *out, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int grid = grid_for((n + 255) / 256, 16);
+    philox_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(ctr), n, philox_keys(seed),
+                                        reinterpret_cast<uint4 *>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_box_muller(const uint32_t *words, int64_t n_pairs, float *z, cudaStream_t st) {
+    if (n_pairs <= 0) return cudaSuccess;
+    const int grid = grid_for((n_pairs + 255) / 256, 16);
+    box_muller_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint2 *>(words), n_pairs,
+                                            reinterpret_cast<float2 *>(z));
+    return cudaGetLastError();
 }
 
 }  // namespace tdm
