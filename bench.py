@@ -62,6 +62,30 @@ def alu_peak_ops(sms: int = 148, clock_ghz: float = 1.965) -> float:
     return sms * 128 * clock_ghz * 1e9
 
 
+RUN_SOURCES = ["tiled_distance_maps_b200/csrc/sampler.cu", "tiled_distance_maps_b200/csrc/common.cuh",
+               "tiled_distance_maps_b200/csrc/internal.h"]
+
+
+def profiled_traffic(summary: str, sources) -> int | None:
+    """DRAM bytes per launch recorded by an ncu capture in profiles/, or None
+    when the kernel's sources have changed since that capture."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    sha = re.search(r"source_sha256: (\w+)", text)
+    nbytes = re.search(r"dram_bytes_per_launch: (\d+)", text)
+    if not sha or not nbytes:
+        return None
+    h = hashlib.sha256()
+    for f in sources:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return int(nbytes.group(1)) if h.hexdigest()[:16] == sha.group(1) else None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -196,14 +220,18 @@ def _config(world):
 def run_ours(args, rank, world, local_rank):
     import torch
     import tiled_distance_maps_b200 as tdm
+    from tiled_distance_maps_b200.parallel import shard_tiling, sharded_seam_discrepancy
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = WORKLOAD
     B, T, S = wl.B, wl.T, wl.S
     n_maps = wl.n_maps
-    tiling = tdm.Tiling(C=1, T=T, B=B, overlap=wl.overlap, sync_every=wl.sync_every,
-                        B_total=B * world, b_offset=B * rank)
+    # one joint run of B * world samples; this rank holds samples
+    # [B * rank, B * (rank + 1)) of every tile
+    tiling = shard_tiling(tdm.Tiling(C=1, T=T, B=B * world, overlap=wl.overlap, sync_every=wl.sync_every),
+                          rank, world)
+    assert tiling.B == B
     ctx = tdm.context(local_rank)
     sched = tdm.Schedule(S, wl.eta, ctx=ctx)
     x0_host = torch.from_numpy(synth.chain_x0(wl.seed, 1, T, sigma=wl.sigma)).contiguous()
@@ -225,10 +253,7 @@ def run_ours(args, rank, world, local_rank):
             ev_run[2 * i_timed + 1].record(stream)
         tdm.mds_recover(maps, n_maps, coords, eig, ctx=ctx)
         tdm.pairwise_dist(coords, n_maps, rec, ctx=ctx)
-        tdm.seam_overlap_sums(rec, tiling, sums, ctx=ctx)
-        if world > 1:
-            torch.distributed.all_reduce(sums)
-        tdm.seam_discrepancy_finalize(sums, tiling, disc, ctx=ctx)
+        sharded_seam_discrepancy(rec, tiling, sums, disc, ctx=ctx)
 
     launches_per_step = 1 + 1 + 1 + (2 if _seam_chunks(T - 1, B) > 1 else 1) + 1
 
@@ -295,7 +320,8 @@ def run_ours(args, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": _config(world),
             "roofline": {"kernel": "ddim_run_kernel", "bound": "alu", "achieved": achieved / 1e12,
-                         "peak": peak / 1e12, "unit": "Tops/s", "frac": achieved / peak, "traffic": None,
+                         "peak": peak / 1e12, "unit": "Tops/s", "frac": achieved / peak,
+                         "traffic": profiled_traffic("ddim_run_kernel_chain32_b1000_cfg.md", RUN_SOURCES),
                          "peak_kind": "derived: 148 SMs x 128 lanes x max SM clock",
                          "ms_per_launch": run_avg_ms,
                          "ops_per_launch": ops},
