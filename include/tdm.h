@@ -228,6 +228,39 @@ tdm_status tdm_seam_overlap_sums(tdm_ctx *ctx, const float *maps, const tdm_tili
 tdm_status tdm_seam_discrepancy_finalize(tdm_ctx *ctx, const float *sums, const tdm_tiling *tiling,
                                          float *out, tdm_stream stream);
 
+/* ---- the same without allocation -------------------------------------------
+ * No counterpart in the paper: this entry point exists for callers that cannot
+ * call cudaMalloc -- an application whose device memory is all handed to its
+ * own pool or arena, a plugin host that forbids allocations outside its own
+ * allocator, or a pipeline that cannot afford the synchronisation that
+ * cudaMalloc/cudaFree may imply.  It needs no tdm_ctx (creating one allocates).
+ *
+ * Computes exactly what tdm_seam_discrepancy computes (out: device [C][T-1];
+ * maps: device [C][T][B][64][64]; both caller-owned, 16-byte aligned), on the
+ * caller's current CUDA device and stream, and calls no cudaMalloc, cudaFree or
+ * allocating routine.  When the samples of a seam are split into chunks, the
+ * partial sums live in one fixed device array of TDM_NOALLOC_SCRATCH_FLOATS
+ * floats (1 MiB) compiled into the library: every GPU that loads the library
+ * holds it until the process exits.  The first call that needs it on a device
+ * looks up its device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before any stream capture.
+ *
+ * All calls on a device share that array and it keeps the last call's partial
+ * sums; each call writes every partial sum it reads before reading it, so no
+ * clearing is needed, but calls that overlap on the GPU (on different streams,
+ * or from different host threads without ordering) race on it and must be
+ * serialised by the caller.
+ *
+ * Errors: TDM_EINVAL (NULL or misaligned pointers, T < 2, B < 1, overlap
+ * outside [1, 32], bad shard fields), TDM_EUNSUPPORTED when the partial sums
+ * would exceed TDM_NOALLOC_SCRATCH_FLOATS (seams x chunks x overlap^2; never
+ * for overlaps up to 16) or the device index is 64 or more, TDM_ECUDA on a
+ * failed launch or symbol lookup.  There is no context to hold an error
+ * message. */
+#define TDM_NOALLOC_SCRATCH_FLOATS 262144
+tdm_status tdm_seam_discrepancy_noalloc(const float *maps, const tdm_tiling *tiling, float *out,
+                                        tdm_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -61,6 +61,7 @@ _SIGS = {
     "tdm_seam_discrepancy_finalize": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp]),
     "tdm_philox4x32": (_i32, [_vp, _vp, _i64, _u64, _vp, _vp]),
     "tdm_box_muller": (_i32, [_vp, _vp, _i64, _vp, _vp]),
+    "tdm_seam_discrepancy_noalloc": (_i32, [_vp, _P(CTiling), _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -322,6 +323,22 @@ def seam_discrepancy_finalize(sums, tiling: Tiling, out, ctx: Context | None = N
     ct = tiling.c()
     ctx.check(_lib.tdm_seam_discrepancy_finalize(ctx.handle, _ptr(sums, "sums", ctx), ctypes.byref(ct),
                                                  _ptr(out, "out", ctx), _stream(ctx)))
+    return out
+
+
+def seam_discrepancy_noalloc(maps, tiling: Tiling, out):
+    """Eq. (6) like seam_discrepancy, for callers that cannot allocate device
+    memory: no context, partial sums in the library's fixed device array (see
+    tdm_seam_discrepancy_noalloc in include/tdm.h).  Runs on the current
+    device and stream; calls that overlap on the GPU race on that array."""
+    import torch
+    _need(maps, tiling.n_maps * 4096, "maps")
+    _need(out, tiling.C * max(tiling.T - 1, 0), "out")
+    ct = tiling.c()
+    stream = _vp(torch.cuda.current_stream(maps.device.index).cuda_stream)
+    st = _lib.tdm_seam_discrepancy_noalloc(_ptr(maps, "maps"), ctypes.byref(ct), _ptr(out, "out"), stream)
+    if st != OK:
+        raise TdmError(st, "tdm_seam_discrepancy_noalloc")
     return out
 
 
