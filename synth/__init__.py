@@ -127,6 +127,11 @@ def cloud_block(seed: int, block: int, noise: float = 0.01):
     return (d * f).astype(np.float32), pts, sig
 
 
+def cloud_block_maps(block: int, seed: int = 0, noise: float = 0.01):
+    """``(block, maps)`` of one block (for process pools)."""
+    return block, cloud_block(seed, block, noise)[0]
+
+
 def cloud_maps(seed: int, start: int, count: int, noise: float = 0.01) -> np.ndarray:
     """Maps ``[start, start+count)`` of the point-cloud recovery workload."""
     out = np.empty((count, N_BEADS, N_BEADS), dtype=np.float32)
