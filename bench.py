@@ -300,6 +300,26 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e2e_ms = e_start.elapsed_time(e_stop)
 
+    # the per-step path (the kernel a real model would drive: eps materialised
+    # by the model, here by the stand-in), timed on its own after the step:
+    # one DDIM step over the same 32,000 maps with CFG w = 1 streams
+    # 64 KiB per map (x, eps_c, eps_u read; x written)
+    ec, eu = torch.empty_like(maps), torch.empty_like(maps)
+    tdm.eps_standin(sched, S - 1, maps, x0, wl.s_c, tdm.STREAM_EPS_C, wl.seed, tiling, ec, ctx=ctx)
+    tdm.eps_standin(sched, S - 1, maps, x0, wl.s_u, tdm.STREAM_EPS_U, wl.seed, tiling, eu, ctx=ctx)
+    n_ps = 20
+    ps_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_ps)]
+    untiled = tdm.Tiling(C=1, T=1, B=n_maps)   # the update alone, no projection launch
+    for i in range(3):
+        tdm.ddim_step(sched, S - 1, maps, ec, eu, wl.w, wl.seed, untiled, ctx=ctx)
+    for i in range(n_ps):
+        ps_ev[2 * i].record(stream)
+        tdm.ddim_step(sched, S - 1 - (i % (S - 1)), maps, ec, eu, wl.w, wl.seed, untiled, ctx=ctx)
+        ps_ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize()
+    step_ms = float(np.median([ps_ev[2 * i].elapsed_time(ps_ev[2 * i + 1]) for i in range(n_ps)]))
+    del ec, eu
+
     t = torch.tensor([ms, e2e_ms, float(np.mean(run_ms))], device=dev, dtype=torch.float64)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -330,6 +350,13 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": x0_host.numel() * 4,
                     "d2h_bytes_per_step": (n_maps * 195 + (T - 1)) * 4},
             "gpu_launches": launches_per_step * args.steps,
+            "per_step_path": {"kernel": "ddim_step_kernel", "bound": "hbm", "ms_per_launch": step_ms,
+                              "bytes_per_launch": n_maps * 4 * 4096 * 4,
+                              "achieved": n_maps * 4 * 4096 * 4 / (step_ms / 1e3) / 1e9,
+                              "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                              "frac": n_maps * 4 * 4096 * 4 / (step_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
+                              "note": "one DDIM step of 32,000 maps, CFG w=1: read x, eps_c, eps_u, write x "
+                                      "(64 KiB per map); timed separately from the step above"},
             "mds_not_converged": bool(flags & tdm.FLAG_MDS_NOT_CONVERGED),
             "peaks": kind,
         }

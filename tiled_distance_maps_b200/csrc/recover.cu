@@ -5,45 +5,49 @@
 // reading used is classical MDS: B = -1/2 J (D*D) J, the top three eigenpairs,
 // x_k = v_k sqrt(max(l_k, 0)).
 //
-// Per map, one warp stages D in shared memory, forms B (lane l computes rows l
-// and l+32 in registers, then writes them over D) and finds the top eigenpairs by subspace iteration on four vectors with a
-// Rayleigh-Ritz step (a 4 x 4 Jacobi eigen-solve) every iteration, stopping when
-// the residual of the three leading Ritz pairs is below kTol * |l_1|.
+// Per map, one warp stages D in shared memory and forms B in place.  The top eigenpairs come from subspace iteration on three
+// vectors with a Rayleigh-Ritz step (a 3 x 3 Jacobi eigen-solve) every
+// iteration, stopping when the residual of the three Ritz pairs is below
+// kTol * |l_1|.  The start basis is the three columns of B with the largest
+// diagonal entries (the points farthest from the centroid): for an exact
+// Euclidean map they already span the answer.  Row l of B stays in registers
+// for the products; row l+32 is read from shared memory.
 #include "common.cuh"
 
 namespace tdm {
 namespace {
 
 constexpr int kMdsWarps = 4;
-constexpr int kLd = kN + 1;       // smem row stride: conflict-free row and column reads
-constexpr int kMaxIt = 32;
+constexpr int kLd = kN + 4;       // smem row stride: 16-byte rows; row float4 and column reads conflict-free
+constexpr int kK = 3;             // subspace dimension
+constexpr int kMaxIt = 48;
 constexpr float kTol = 4e-6f;
-
-// start vectors: column c of V0 has entry (-1)^bit_j(v0_mask(c))
-__host__ __device__ constexpr unsigned long long v0_mask(int c) {
-    return c == 0 ? 0x9E3779B97F4A7C15ull : c == 1 ? 0xBF58476D1CE4E5B9ull
-         : c == 2 ? 0x94D049BB133111EBull : 0xD6E8FEB86659FD93ull;
-}
 
 __device__ __forceinline__ float wsum(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
     return v;
 }
-__device__ __forceinline__ float wmax(float v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-    return v;
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float rsqrt_approx(float x) {
+    float r;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
-// Gram-Schmidt applied twice per column ("twice is enough") on 64 x 4 columns
-// held as rows (l, l+32) per lane.
-__device__ __forceinline__ void orthonormalize(float (&a0)[4], float (&a1)[4]) {
+// Gram-Schmidt applied twice per column ("twice is enough") on 64 x kK
+// columns held as rows (l, l+32) per lane.
+__device__ __forceinline__ void orthonormalize(float (&a0)[kK], float (&a1)[kK]) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < kK; ++c) {
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass) {
-            float d[4];
+            float d[kK];
 #pragma unroll
             for (int p = 0; p < c; ++p) d[p] = wsum(fmaf(a0[p], a0[c], a1[p] * a1[c]));
 #pragma unroll
@@ -53,48 +57,50 @@ __device__ __forceinline__ void orthonormalize(float (&a0)[4], float (&a1)[4]) {
             }
         }
         const float nn = wsum(fmaf(a0[c], a0[c], a1[c] * a1[c]));
-        const float inv = nn > 0.0f ? 1.0f / sqrtf(nn) : 0.0f;
+        const float inv = nn > 1e-37f ? rsqrt_approx(nn) : 0.0f;
         a0[c] *= inv;
         a1[c] *= inv;
     }
 }
 
+// One Jacobi rotation zeroing H[P][Q] of the symmetric kK x kK H (both
+// halves kept), accumulated into Y (Golub & Van Loan §8.5: the symmetric 2 x 2
+// Schur step, with the diagonal updated by t * H[P][Q]).
 template <int P, int Q>
-__device__ __forceinline__ void jrot(float (&H)[4][4], float (&Y)[4][4]) {
+__device__ __forceinline__ void jrot(float (&H)[kK][kK], float (&Y)[kK][kK]) {
     const float apq = H[P][Q];
-    if (apq == 0.0f) return;
-    const float tau = (H[Q][Q] - H[P][P]) / (2.0f * apq);
-    const float t = copysignf(1.0f, tau) / (fabsf(tau) + sqrtf(fmaf(tau, tau, 1.0f)));
-    const float c = 1.0f / sqrtf(fmaf(t, t, 1.0f));
+    if (!(fabsf(apq) > 1e-9f * (fabsf(H[P][P]) + fabsf(H[Q][Q])))) return;
+    const float theta = (H[Q][Q] - H[P][P]) * 0.5f * rcp_approx(apq);
+    const float r2 = fmaf(theta, theta, 1.0f);
+    const float t = copysignf(rcp_approx(fabsf(theta) + r2 * rsqrt_approx(r2)), theta);
+    const float c = rsqrt_approx(fmaf(t, t, 1.0f));
     const float s = t * c;
+    H[P][P] = fmaf(-t, apq, H[P][P]);
+    H[Q][Q] = fmaf(t, apq, H[Q][Q]);
+    H[P][Q] = H[Q][P] = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kK; ++k) {
+        if (k == P || k == Q) continue;
         const float hp = H[k][P], hq = H[k][Q];
-        H[k][P] = c * hp - s * hq;
-        H[k][Q] = s * hp + c * hq;
+        H[k][P] = H[P][k] = fmaf(c, hp, -s * hq);
+        H[k][Q] = H[Q][k] = fmaf(s, hp, c * hq);
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float hp = H[P][k], hq = H[Q][k];
-        H[P][k] = c * hp - s * hq;
-        H[Q][k] = s * hp + c * hq;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kK; ++k) {
         const float yp = Y[k][P], yq = Y[k][Q];
-        Y[k][P] = c * yp - s * yq;
-        Y[k][Q] = s * yp + c * yq;
+        Y[k][P] = fmaf(c, yp, -s * yq);
+        Y[k][Q] = fmaf(s, yp, c * yq);
     }
 }
 
 template <int I, int J>
-__device__ __forceinline__ void sort_pair(float (&th)[4], float (&Y)[4][4]) {
+__device__ __forceinline__ void sort_pair(float (&th)[kK], float (&Y)[kK][kK]) {
     if (th[I] < th[J]) {
         const float tt = th[I];
         th[I] = th[J];
         th[J] = tt;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < kK; ++k) {
             const float y = Y[k][I];
             Y[k][I] = Y[k][J];
             Y[k][J] = y;
@@ -102,43 +108,51 @@ __device__ __forceinline__ void sort_pair(float (&th)[4], float (&Y)[4][4]) {
     }
 }
 
-// Cyclic Jacobi on a symmetric 4 x 4 matrix (Golub & Van Loan §8.5); eigenvalues
-// sorted in descending order, eigenvectors in the columns of Y.
-__device__ __forceinline__ void eig4(float (&H)[4][4], float (&Y)[4][4], float (&th)[4]) {
+// Cyclic Jacobi on a symmetric 3 x 3 matrix; eigenvalues sorted in descending
+// order, eigenvectors in the columns of Y.
+__device__ __forceinline__ void eig3(float (&H)[kK][kK], float (&Y)[kK][kK], float (&th)[kK]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kK; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) Y[i][j] = i == j ? 1.0f : 0.0f;
-    for (int sweep = 0; sweep < 10; ++sweep) {
-        const float off = H[0][1] * H[0][1] + H[0][2] * H[0][2] + H[0][3] * H[0][3] + H[1][2] * H[1][2] +
-                          H[1][3] * H[1][3] + H[2][3] * H[2][3];
-        const float dia = H[0][0] * H[0][0] + H[1][1] * H[1][1] + H[2][2] * H[2][2] + H[3][3] * H[3][3];
+        for (int j = 0; j < kK; ++j) Y[i][j] = i == j ? 1.0f : 0.0f;
+    for (int sweep = 0; sweep < 12; ++sweep) {
+        const float off = H[0][1] * H[0][1] + H[0][2] * H[0][2] + H[1][2] * H[1][2];
+        const float dia = H[0][0] * H[0][0] + H[1][1] * H[1][1] + H[2][2] * H[2][2];
         if (off <= 1e-14f * dia) break;
         jrot<0, 1>(H, Y);
         jrot<0, 2>(H, Y);
-        jrot<0, 3>(H, Y);
         jrot<1, 2>(H, Y);
-        jrot<1, 3>(H, Y);
-        jrot<2, 3>(H, Y);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) th[i] = H[i][i];
+    for (int i = 0; i < kK; ++i) th[i] = H[i][i];
     sort_pair<0, 1>(th, Y);
-    sort_pair<2, 3>(th, Y);
-    sort_pair<0, 2>(th, Y);
-    sort_pair<1, 3>(th, Y);
     sort_pair<1, 2>(th, Y);
+    sort_pair<0, 1>(th, Y);
+}
+
+// (value, index) of the warp-wide maximum; ties go to the lower index.
+__device__ __forceinline__ void warp_argmax(float &v, int &i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, off);
+        if (ov > v || (ov == v && oi < i)) {
+            v = ov;
+            i = oi;
+        }
+    }
 }
 
 __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__restrict__ maps, int64_t n,
-                                                             float *__restrict__ coords,
-                                                             float *__restrict__ eig,
-                                                             uint32_t *__restrict__ flags) {
-    extern __shared__ float smem[];
+                                                                float *__restrict__ coords,
+                                                                float *__restrict__ eig,
+                                                                uint32_t *__restrict__ flags) {
+    extern __shared__ __align__(16) float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float *sD = smem + warp * (kN * kLd);
     float4 *sV = reinterpret_cast<float4 *>(smem + kMdsWarps * kN * kLd) + warp * kN;
     float *sR = smem + kMdsWarps * kN * kLd + kMdsWarps * kN * 4 + warp * kN;
+    const int i0 = lane, i1 = lane + 32;
 
     for (int64_t m = (int64_t)blockIdx.x * kMdsWarps + warp; m < n; m += (int64_t)gridDim.x * kMdsWarps) {
         const float *D = maps + m * kMapFloats;
@@ -146,116 +160,139 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         for (int it = 0; it < 32; ++it) {
             const int idx = it * 32 + lane;
             const int row = idx >> 4, c4 = (idx & 15) << 2;
-            const float4 v = __ldcs(reinterpret_cast<const float4 *>(D + row * kN + c4));
-            float *dst = sD + row * kLd + c4;
-            dst[0] = v.x;
-            dst[1] = v.y;
-            dst[2] = v.z;
-            dst[3] = v.w;
+            *reinterpret_cast<float4 *>(sD + row * kLd + c4) =
+                __ldcs(reinterpret_cast<const float4 *>(D + row * kN + c4));
         }
         __syncwarp();
 
-        // symmetrise and square; lane holds rows lane and lane+32
-        float b0[kN], b1[kN];
-        float mx = 0.0f;
+        // e_ij = D_ij + D_ji (twice the symmetric part); S = (e/2)^2, so
+        // B = -1/2 J S J = -1/8 J (e*e) J.  Each unordered pair {v, w} is
+        // read and written by one lane only (virtual lane v in {l, l+32} takes
+        // w = v + k mod 64 for k = 0..32, and k = 32 only for v < 32), so e*e
+        // replaces D at (v, w) and (w, v) with no barrier between the reads
+        // and the writes; banks (5 l + k) and (5 l + 4 k) mod 32 are distinct
+        // over the lanes.
+#pragma unroll 3
+        for (int k = 0; k <= 32; ++k) {
 #pragma unroll
-        for (int j = 0; j < kN; ++j) {
-            const float d0 = 0.5f * (sD[lane * kLd + j] + sD[j * kLd + lane]);
-            const float d1 = 0.5f * (sD[(lane + 32) * kLd + j] + sD[j * kLd + lane + 32]);
-            b0[j] = d0 * d0;
-            b1[j] = d1 * d1;
-            mx = fmaxf(mx, fmaxf(b0[j], b1[j]));
+            for (int h = 0; h < 2; ++h) {
+                if (k == 32 && h == 1) continue;
+                const int v = lane + 32 * h;
+                const int w = (v + k) & (kN - 1);
+                const float e = sD[v * kLd + w] + sD[w * kLd + v];
+                const float e2 = e * e;
+                sD[v * kLd + w] = e2;
+                sD[w * kLd + v] = e2;
+            }
         }
-        // exact power-of-two rescale of D*D to O(1), undone on the eigenvalues
-        mx = wmax(mx);
-        int ex = 0;
-        frexpf(mx, &ex);
-        const float scale = mx > 0.0f && isfinite(mx) ? ldexpf(1.0f, -ex) : 1.0f;
+        __syncwarp();
+        // row means of e*e (lane: rows i0 and i1), grand mean
         float rs0 = 0.0f, rs1 = 0.0f;
-#pragma unroll
-        for (int j = 0; j < kN; ++j) {
-            b0[j] *= scale;
-            b1[j] *= scale;
-            rs0 += b0[j];
-            rs1 += b1[j];
+#pragma unroll 4
+        for (int j4 = 0; j4 < kN / 4; ++j4) {
+            const float4 a = *reinterpret_cast<const float4 *>(sD + i0 * kLd + 4 * j4);
+            const float4 b = *reinterpret_cast<const float4 *>(sD + i1 * kLd + 4 * j4);
+            rs0 += (a.x + a.y) + (a.z + a.w);
+            rs1 += (b.x + b.y) + (b.z + b.w);
         }
         const float r0 = rs0 * (1.0f / kN), r1 = rs1 * (1.0f / kN);
         const float gm = wsum(r0 + r1) * (1.0f / kN);
+        // exact power-of-two scale bringing the mean of e*e to O(1); undone on
+        // the eigenvalues
+        int ex = 0;
+        frexpf(gm, &ex);
+        const float scale = gm > 0.0f && isfinite(gm) ? ldexpf(1.0f, -ex) : 1.0f;
+        const float cs = -0.125f * scale;
+        sR[i0] = r0;
+        sR[i1] = r1;
         __syncwarp();
-        sR[lane] = r0;
-        sR[lane + 32] = r1;
-        __syncwarp();
-        // double centring: B_ij = -1/2 (D2_ij - r_i - r_j + g)
+        // double centring in place, row by row: B_ij = cs (e2_ij - r_i - r_j + g);
+        // row i0 of B is also kept in registers for the products
+        const float g0 = gm - r0, g1 = gm - r1;
+        float b0[kN];
 #pragma unroll
-        for (int j = 0; j < kN; ++j) {
-            const float rj = sR[j];
-            b0[j] = -0.5f * (b0[j] - r0 - rj + gm);
-            b1[j] = -0.5f * (b1[j] - r1 - rj + gm);
+        for (int j4 = 0; j4 < kN / 4; ++j4) {
+            const float4 rj = *reinterpret_cast<const float4 *>(sR + 4 * j4);
+            float4 a = *reinterpret_cast<const float4 *>(sD + i0 * kLd + 4 * j4);
+            float4 b = *reinterpret_cast<const float4 *>(sD + i1 * kLd + 4 * j4);
+            a.x = cs * ((a.x + g0) - rj.x);
+            a.y = cs * ((a.y + g0) - rj.y);
+            a.z = cs * ((a.z + g0) - rj.z);
+            a.w = cs * ((a.w + g0) - rj.w);
+            b.x = cs * ((b.x + g1) - rj.x);
+            b.y = cs * ((b.y + g1) - rj.y);
+            b.z = cs * ((b.z + g1) - rj.z);
+            b.w = cs * ((b.w + g1) - rj.w);
+            b0[4 * j4] = a.x;
+            b0[4 * j4 + 1] = a.y;
+            b0[4 * j4 + 2] = a.z;
+            b0[4 * j4 + 3] = a.w;
+            *reinterpret_cast<float4 *>(sD + i0 * kLd + 4 * j4) = a;
+            *reinterpret_cast<float4 *>(sD + i1 * kLd + 4 * j4) = b;
         }
+        __syncwarp();
 
-        // first basis: orth(B V0), from the register copy of B's rows
-        float v0[4] = {0.f, 0.f, 0.f, 0.f}, v1[4] = {0.f, 0.f, 0.f, 0.f};
+        // start basis: the columns of the kK largest diagonal entries
+        float v0[kK], v1[kK];
+        {
+            float d0 = sD[i0 * kLd + i0], d1 = sD[i1 * kLd + i1];
 #pragma unroll
-        for (int j = 0; j < kN; ++j)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if ((v0_mask(c) >> j) & 1ull) {
-                    v0[c] -= b0[j];
-                    v1[c] -= b1[j];
-                } else {
-                    v0[c] += b0[j];
-                    v1[c] += b1[j];
-                }
+            for (int c = 0; c < kK; ++c) {
+                float bv = d0 >= d1 ? d0 : d1;
+                int bi = d0 >= d1 ? i0 : i1;
+                warp_argmax(bv, bi);
+                if (bi == i0) d0 = -INFINITY;
+                if (bi == i1) d1 = -INFINITY;
+                v0[c] = sD[bi * kLd + i0];     // B[i0][bi] = B[bi][i0]
+                v1[c] = sD[bi * kLd + i1];
             }
-        // B replaces D in shared memory (every lane has finished reading D)
-#pragma unroll
-        for (int j = 0; j < kN; ++j) {
-            sD[lane * kLd + j] = b0[j];
-            sD[(lane + 32) * kLd + j] = b1[j];
         }
         orthonormalize(v0, v1);
-        sV[lane] = make_float4(v0[0], v0[1], v0[2], v0[3]);
-        sV[lane + 32] = make_float4(v1[0], v1[1], v1[2], v1[3]);
+        sV[i0] = make_float4(v0[0], v0[1], v0[2], 0.0f);
+        sV[i1] = make_float4(v1[0], v1[1], v1[2], 0.0f);
 
-        float th[4] = {0.f, 0.f, 0.f, 0.f};
-        float u0[4], u1[4];
+        float th[kK] = {0.f, 0.f, 0.f};
+        float u0[kK], u1[kK];
         bool conv = false;
-        const float *bl = sD + lane * kLd, *bh = sD + (lane + 32) * kLd;
+        const float *bh = sD + i1 * kLd;
         for (int it = 0; it < kMaxIt; ++it) {
             __syncwarp();
-            float w0[4] = {0.f, 0.f, 0.f, 0.f}, w1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-            for (int j = 0; j < kN; ++j) {
-                const float4 v = sV[j];
-                const float x0 = bl[j], x1 = bh[j];
-                w0[0] = fmaf(x0, v.x, w0[0]);
-                w0[1] = fmaf(x0, v.y, w0[1]);
-                w0[2] = fmaf(x0, v.z, w0[2]);
-                w0[3] = fmaf(x0, v.w, w0[3]);
-                w1[0] = fmaf(x1, v.x, w1[0]);
-                w1[1] = fmaf(x1, v.y, w1[1]);
-                w1[2] = fmaf(x1, v.z, w1[2]);
-                w1[3] = fmaf(x1, v.w, w1[3]);
+            float w0[kK] = {0.f, 0.f, 0.f}, w1[kK] = {0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j4 = 0; j4 < kN / 4; ++j4) {
+                const float4 x1 = *reinterpret_cast<const float4 *>(bh + 4 * j4);
+                const float xb[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const float4 v = sV[4 * j4 + t];
+                    const float xa = b0[4 * j4 + t];
+                    w0[0] = fmaf(xa, v.x, w0[0]);
+                    w0[1] = fmaf(xa, v.y, w0[1]);
+                    w0[2] = fmaf(xa, v.z, w0[2]);
+                    w1[0] = fmaf(xb[t], v.x, w1[0]);
+                    w1[1] = fmaf(xb[t], v.y, w1[1]);
+                    w1[2] = fmaf(xb[t], v.z, w1[2]);
+                }
             }
             // Rayleigh quotient H = V^T B V (symmetrised)
-            float H[4][4];
+            float H[kK][kK];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < kK; ++a)
 #pragma unroll
-                for (int b = a; b < 4; ++b) {
+                for (int b = a; b < kK; ++b) {
                     const float h = 0.5f * wsum(fmaf(v0[a], w0[b], fmaf(v0[b], w0[a],
                                                      fmaf(v1[a], w1[b], v1[b] * w1[a]))));
                     H[a][b] = h;
                     H[b][a] = h;
                 }
-            float Y[4][4];
-            eig4(H, Y, th);
-            float bu0[4], bu1[4];
+            float Y[kK][kK];
+            eig3(H, Y, th);
+            float bu0[kK], bu1[kK];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kK; ++c) {
                 u0[c] = u1[c] = bu0[c] = bu1[c] = 0.0f;
 #pragma unroll
-                for (int a = 0; a < 4; ++a) {
+                for (int a = 0; a < kK; ++a) {
                     u0[c] = fmaf(v0[a], Y[a][c], u0[c]);
                     u1[c] = fmaf(v1[a], Y[a][c], u1[c]);
                     bu0[c] = fmaf(w0[a], Y[a][c], bu0[c]);
@@ -264,7 +301,7 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
             }
             float rmax = 0.0f;
 #pragma unroll
-            for (int c = 0; c < 3; ++c) {
+            for (int c = 0; c < kK; ++c) {
                 const float e0 = fmaf(-th[c], u0[c], bu0[c]);
                 const float e1 = fmaf(-th[c], u1[c], bu1[c]);
                 rmax = fmaxf(rmax, wsum(fmaf(e0, e0, e1 * e1)));
@@ -276,23 +313,23 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
             }
             orthonormalize(bu0, bu1);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kK; ++c) {
                 v0[c] = bu0[c];
                 v1[c] = bu1[c];
             }
             __syncwarp();
-            sV[lane] = make_float4(v0[0], v0[1], v0[2], v0[3]);
-            sV[lane + 32] = make_float4(v1[0], v1[1], v1[2], v1[3]);
+            sV[i0] = make_float4(v0[0], v0[1], v0[2], 0.0f);
+            sV[i1] = make_float4(v1[0], v1[1], v1[2], 0.0f);
         }
         if (!conv && lane == 0) atomicOr(flags, (uint32_t)TDM_FLAG_MDS_NOT_CONVERGED);
 
         const float inv_scale = 1.0f / scale;
         float *X = coords + m * (kN * 3);
 #pragma unroll
-        for (int c = 0; c < 3; ++c) {
+        for (int c = 0; c < kK; ++c) {
             const float sq = sqrtf(fmaxf(th[c], 0.0f) * inv_scale);
-            X[lane * 3 + c] = u0[c] * sq;
-            X[(lane + 32) * 3 + c] = u1[c] * sq;
+            X[i0 * 3 + c] = u0[c] * sq;
+            X[i1 * 3 + c] = u1[c] * sq;
         }
         if (eig != nullptr && lane < 3) eig[m * 3 + lane] = (lane == 0 ? th[0] : lane == 1 ? th[1] : th[2]) * inv_scale;
         __syncwarp();
@@ -337,6 +374,7 @@ cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigva
                        cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
     const size_t smem = sizeof(float) * (size_t)kMdsWarps * (kN * kLd + kN * 4 + kN);
+    static_assert((kMdsWarps * kN * kLd * sizeof(float)) % 16 == 0, "float4 alignment of the V tiles");
     cudaError_t e = cudaFuncSetAttribute(mds_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
