@@ -180,6 +180,21 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
  * [0, o); M is written to both.  Idempotent.  1 <= overlap <= 32. */
 tdm_status tdm_seam_project(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, tdm_stream stream);
 
+/* ---- stitching ------------------------------------------------------------
+ * Kabsch stitching of per-tile coordinates into chains (ParaChromo §4.3.2 last
+ * paragraph; §5.5, Fig. 4).  coords: device [C][T][B][64][3] (tile k, sample b
+ * of chain c; e.g. tdm_mds_recover's output of a tiled batch).  For every seam,
+ * tile k+1 is mapped onto tile k by x -> R x + t with R the orthogonal polar
+ * factor of the cross-covariance of the o shared beads (an improper R is
+ * allowed: recovered coordinates are defined up to reflection), t matching the
+ * centroids; the maps compose along the chain so every tile lands in tile 0's
+ * frame.  chain_out: device [C][B][L][3], L = 64 + (T-1)(64-o); an overlap
+ * bead is the mean of its two aligned copies.  residual_out: device
+ * [C][B][T-1] (may be NULL), the RMSD over the o beads of each seam after the
+ * alignment, in the coordinates' units.  Needs overlap >= 3 when T > 1. */
+tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling *tiling, float *chain_out,
+                             float *residual_out, tdm_stream stream);
+
 /* ---- noise primitives ----------------------------------------------------
  * The two stages of every noise stream, on caller data, so that a caller can
  * reproduce any noise value and check the transform's error exhaustively. */

@@ -146,6 +146,49 @@ def cloud_maps(seed: int, start: int, count: int, noise: float = 0.01) -> np.nda
     return out
 
 
+def random_orthogonal(g: np.random.Generator, proper: bool = False) -> np.ndarray:
+    """A random 3x3 orthogonal matrix (det -1 half of the time unless proper)."""
+    q, r = np.linalg.qr(g.standard_normal((3, 3)))
+    q = q * np.sign(np.diag(r))
+    if proper and np.linalg.det(q) < 0:
+        q[:, 0] = -q[:, 0]
+    return q
+
+
+def tile_coords(seed: int, n_chains: int, n_tiles: int, n_samples: int, overlap: int = OVERLAP,
+                noise: float = 0.0, proper: bool = False):
+    """Per-tile coordinates ``[C][T][B][64][3]`` (float32) of random-walk chains.
+
+    Sample b of chain c is one walk of the chain's length; tile k holds beads
+    [k*stride, k*stride + 64) under its own random orthogonal map (improper
+    half of the time unless ``proper``) and translation, plus ``noise`` N(0,1)
+    per coordinate -- the shape of per-tile recovered coordinates.  Also
+    returns the walks ``[C][B][L][3]`` (float64) and the tile maps
+    ``(R [C][T][B][3][3], t [C][T][B][3])`` (tile beads = R @ walk + t).
+    """
+    stride = N_BEADS - overlap
+    L = chain_beads(n_tiles, overlap)
+    out = np.empty((n_chains, n_tiles, n_samples, N_BEADS, 3), dtype=np.float32)
+    walks = np.empty((n_chains, n_samples, L, 3))
+    Rs = np.empty((n_chains, n_tiles, n_samples, 3, 3))
+    ts = np.empty((n_chains, n_tiles, n_samples, 3))
+    for c in range(n_chains):
+        for b in range(n_samples):
+            g = _rng(seed, 0x57C4, c, b)
+            steps = g.standard_normal((L - 1, 3))
+            w = np.concatenate([np.zeros((1, 3)), np.cumsum(steps, axis=0)], axis=0)
+            walks[c, b] = w
+            for k in range(n_tiles):
+                R = random_orthogonal(g, proper)
+                t = g.standard_normal(3) * 10.0
+                x = w[k * stride:k * stride + N_BEADS] @ R.T + t
+                if noise:
+                    x = x + noise * g.standard_normal(x.shape)
+                out[c, k, b] = x
+                Rs[c, k, b], ts[c, k, b] = R, t
+    return out, walks, (Rs, ts)
+
+
 def random_points(seed: int, count: int, n: int = N_BEADS, scale: float = 1.0) -> np.ndarray:
     """``[count, n, 3]`` float64 Gaussian points (for exact-distance checks)."""
     return _rng(seed, 0x9017, count, n).standard_normal((count, n, 3)) * scale

@@ -1,0 +1,63 @@
+"""GPU parity of Kabsch stitching against the float64 oracle."""
+import numpy as np
+import pytest
+
+import synth
+from oracle import stitch as ostitch
+from tests.gpu_util import dev, host, needs_gpu, torch
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+# stitched chains, normwise over a chain: float32 polar factors composed over
+# up to 39 seams; residuals relative to the oracle's, with a floor at the
+# larger of 1e-3 of the noise and the float32 rounding of the coordinates
+TOL_CHAIN = 1e-4
+TOL_RESID = 1e-3
+
+
+@pytest.fixture(scope="module")
+def tdm():
+    import tiled_distance_maps_b200 as m
+    return m
+
+
+def _run(tdm, X, T, overlap):
+    C, _, B = X.shape[:3]
+    t = tdm.Tiling(C=C, T=T, B=B, overlap=overlap)
+    L = 64 + (T - 1) * (64 - overlap)
+    chain = torch.empty(C * B * L * 3, device="cuda")
+    res = torch.empty(max(C * B * (T - 1), 1), device="cuda")
+    tdm.kabsch_stitch(dev(X).reshape(-1), t, chain, res if T > 1 else None)
+    torch.cuda.synchronize()
+    return host(chain).reshape(C, B, L, 3), host(res)[:C * B * (T - 1)].reshape(C, B, T - 1)
+
+
+@pytest.mark.parametrize("C,T,B,o,noise", [(2, 5, 3, 12, 0.05), (1, 32, 8, 12, 0.02), (2, 40, 3, 8, 0.05),
+                                           (1, 3, 2, 32, 0.0), (3, 1, 2, 12, 0.0)])
+def test_stitch_matches_oracle(tdm, C, T, B, o, noise):
+    X, _, _ = synth.tile_coords(T * 7 + B, C, T, B, overlap=o, noise=noise)
+    got, res = _run(tdm, X, T, o)
+    ref, rref = ostitch.stitch(X.astype(np.float64), o)
+    scale = np.abs(ref).max(axis=(-1, -2))
+    err = (np.abs(got - ref).max(axis=(-1, -2)) / scale).max()
+    assert err <= TOL_CHAIN, err
+    if T > 1:
+        # noise-free tiles have residual 0 up to float32 rounding of the
+        # coordinates: the floor is that rounding level
+        floor = max(1e-3 * noise, 4e-6 * float(np.abs(X).max()))
+        rel = np.abs(res - rref) / np.maximum(rref, floor)
+        assert rel.max() <= TOL_RESID, rel.max()
+
+
+def test_stitch_chromosome_chain_full_size(tdm):
+    # 32 tiles x 1000 samples: every sample's chain on the GPU, 6 sampled
+    # chains through the oracle
+    C, T, B = 1, 32, 1000
+    X, _, _ = synth.tile_coords(99, C, T, B, noise=0.02)
+    got, res = _run(tdm, X, T, 12)
+    assert np.isfinite(got).all() and np.isfinite(res).all()
+    idx = np.random.default_rng(0).choice(B, size=6, replace=False)
+    ref, rref = ostitch.stitch(X[:, :, idx].astype(np.float64))
+    scale = np.abs(ref).max(axis=(-1, -2))
+    assert (np.abs(got[:, idx] - ref).max(axis=(-1, -2)) / scale).max() <= TOL_CHAIN
+    assert (np.abs(res[:, idx] - rref) / np.maximum(rref, 2e-5)).max() <= TOL_RESID

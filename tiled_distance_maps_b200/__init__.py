@@ -62,6 +62,7 @@ _SIGS = {
     "tdm_philox4x32": (_i32, [_vp, _vp, _i64, _u64, _vp, _vp]),
     "tdm_box_muller": (_i32, [_vp, _vp, _i64, _vp, _vp]),
     "tdm_seam_discrepancy_noalloc": (_i32, [_vp, _P(CTiling), _vp, _vp]),
+    "tdm_kabsch_stitch": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -324,6 +325,22 @@ def seam_discrepancy_finalize(sums, tiling: Tiling, out, ctx: Context | None = N
     ctx.check(_lib.tdm_seam_discrepancy_finalize(ctx.handle, _ptr(sums, "sums", ctx), ctypes.byref(ct),
                                                  _ptr(out, "out", ctx), _stream(ctx)))
     return out
+
+
+def kabsch_stitch(coords, tiling: Tiling, chain_out, residual_out=None, ctx: Context | None = None):
+    """Stitch per-tile coordinates ``[C][T][B][64][3]`` into chains
+    ``[C][B][L][3]`` (L = 64 + (T-1)(64-overlap)); optional per-seam RMSD
+    ``[C][B][T-1]`` (see tdm_kabsch_stitch)."""
+    ctx = ctx or context(coords.device.index)
+    L = 64 + (tiling.T - 1) * (64 - tiling.overlap)
+    _need(coords, tiling.n_maps * 192, "coords")
+    _need(chain_out, tiling.C * tiling.B * L * 3, "chain_out")
+    _need(residual_out, tiling.C * tiling.B * max(tiling.T - 1, 0), "residual_out")
+    ct = tiling.c()
+    ctx.check(_lib.tdm_kabsch_stitch(ctx.handle, _ptr(coords, "coords", ctx), ctypes.byref(ct),
+                                     _ptr(chain_out, "chain_out", ctx), _ptr(residual_out, "residual_out", ctx),
+                                     _stream(ctx)))
+    return chain_out
 
 
 def seam_discrepancy_noalloc(maps, tiling: Tiling, out):

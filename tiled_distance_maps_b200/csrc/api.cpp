@@ -371,6 +371,26 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "ddim_run launch");
 }
 
+// ---- stitching -----------------------------------------------------------------------
+
+tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling *tiling, float *chain_out,
+                             float *residual_out, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    Tiling t;
+    tdm_status s = check_tiling(ctx, tiling, &t);
+    if (s != TDM_OK) return s;
+    if (t.T > 1 && t.overlap < 3) return fail(ctx, TDM_EINVAL, "stitching needs an overlap of at least 3 beads");
+    if (t.n_maps() == 0) return TDM_OK;
+    if ((s = check_maps(ctx, coords, "coords")) != TDM_OK || (s = check_maps(ctx, chain_out, "chain_out")) != TDM_OK)
+        return s;
+    if (residual_out != nullptr && (reinterpret_cast<uintptr_t>(residual_out) & 3u))
+        return fail(ctx, TDM_EINVAL, "residual_out is not 4-byte aligned");
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_stitch(coords, t, chain_out, t.T > 1 ? residual_out : nullptr,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "stitch launch");
+}
+
 // ---- noise primitives ---------------------------------------------------------------
 
 tdm_status tdm_philox4x32(tdm_ctx *ctx, const uint32_t *ctr, int64_t n, uint64_t seed, uint32_t *out,

@@ -70,12 +70,14 @@ __device__ __forceinline__ uint4 noise_counter(int r, int q, uint32_t step_word,
 // and cosine approximations hold their stated error, and the sign is restored:
 // cos(2 pi u2) = -cos(2 pi (u2 - 1/2)), likewise for sin.
 __device__ __forceinline__ float2 box_muller(uint32_t a, uint32_t b) {
-    const float e = __uint_as_float(0x3F800000u | (a >> 9)) - 1.0f;
-    const float u1 = 1.0f - e;
+    const float f = __uint_as_float(0x3F800000u | (a >> 9));     // 1 + e
+    const float e = f - 1.0f;
+    const float u1 = 2.0f - f;
     const float h = __uint_as_float(0x3F800000u | (b >> 9)) - 1.5f;
     float lg, r, sn, cs;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(u1));
-    const float v_log = fmaxf(-1.3862943611198906f * lg, 0.0f);     // -2 ln2 log2 u1
+    // for e >= 2^-6 the log branch is >= 0.03, well clear of its error
+    const float v_log = -1.3862943611198906f * lg;                   // -2 ln2 log2 u1
     const float v_ser = e * fmaf(e, fmaf(e, 0.6666667f, 1.0f), 2.0f);
     const float v = e < 0.015625f ? v_ser : v_log;
     asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));

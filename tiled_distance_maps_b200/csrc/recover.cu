@@ -150,7 +150,11 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
     extern __shared__ __align__(16) float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float *sD = smem + warp * (kN * kLd);
-    float4 *sV = reinterpret_cast<float4 *>(smem + kMdsWarps * kN * kLd) + warp * kN;
+    // V as (c0, c1) pairs and c2 values: a broadcast 64-bit load is served
+    // per half warp and a 32-bit one per warp (3 wavefronts per row of V
+    // against 4 for a 128-bit broadcast)
+    float2 *sV01 = reinterpret_cast<float2 *>(smem + kMdsWarps * kN * kLd) + warp * kN * 2;
+    float *sV2 = reinterpret_cast<float *>(sV01 + kN);
     float *sR = smem + kMdsWarps * kN * kLd + kMdsWarps * kN * 4 + warp * kN;
     const int i0 = lane, i1 = lane + 32;
 
@@ -248,8 +252,10 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
             }
         }
         orthonormalize(v0, v1);
-        sV[i0] = make_float4(v0[0], v0[1], v0[2], 0.0f);
-        sV[i1] = make_float4(v1[0], v1[1], v1[2], 0.0f);
+        sV01[i0] = make_float2(v0[0], v0[1]);
+        sV01[i1] = make_float2(v1[0], v1[1]);
+        sV2[i0] = v0[2];
+        sV2[i1] = v1[2];
 
         float th[kK] = {0.f, 0.f, 0.f};
         float u0[kK], u1[kK];
@@ -264,7 +270,8 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                 const float xb[4] = {x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    const float4 v = sV[4 * j4 + t];
+                    const float2 v01 = sV01[4 * j4 + t];
+                    const float4 v = make_float4(v01.x, v01.y, sV2[4 * j4 + t], 0.0f);
                     const float xa = b0[4 * j4 + t];
                     w0[0] = fmaf(xa, v.x, w0[0]);
                     w0[1] = fmaf(xa, v.y, w0[1]);
@@ -318,8 +325,10 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                 v1[c] = bu1[c];
             }
             __syncwarp();
-            sV[i0] = make_float4(v0[0], v0[1], v0[2], 0.0f);
-            sV[i1] = make_float4(v1[0], v1[1], v1[2], 0.0f);
+            sV01[i0] = make_float2(v0[0], v0[1]);
+            sV01[i1] = make_float2(v1[0], v1[1]);
+            sV2[i0] = v0[2];
+            sV2[i1] = v1[2];
         }
         if (!conv && lane == 0) atomicOr(flags, (uint32_t)TDM_FLAG_MDS_NOT_CONVERGED);
 
