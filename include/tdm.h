@@ -180,6 +180,20 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
  * [0, o); M is written to both.  Idempotent.  1 <= overlap <= 32. */
 tdm_status tdm_seam_project(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, tdm_stream stream);
 
+/* ---- coordinate refinement ----------------------------------------------
+ * SMACOF stress majorisation of coordinates against their maps (ParaChromo
+ * §3.1: distance-geometry initialisation "followed by coordinate refinement";
+ * the method is not on the pages -- read as minimising the raw stress
+ * sum_{i<j} (|x_i - x_j| - D_ij)^2).  maps: device [n][64][64] (symmetrised
+ * as (D + D^T)/2); coords: device [n][64][3], the start (e.g.
+ * tdm_mds_recover's output) on entry, the result on return.  Each of the
+ * `iterations` steps is the Guttman transform x_i <- (1/64) sum_{j != i}
+ * (D_ij / d_ij) (x_i - x_j) (terms with d_ij = 0 left out), which never
+ * increases the stress.  stress_out (device [n], may be NULL) receives the
+ * final stress. */
+tdm_status tdm_refine_smacof(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, int32_t iterations,
+                             float *stress_out, tdm_stream stream);
+
 /* ---- stitching ------------------------------------------------------------
  * Kabsch stitching of per-tile coordinates into chains (ParaChromo §4.3.2 last
  * paragraph; §5.5, Fig. 4).  coords: device [C][T][B][64][3] (tile k, sample b

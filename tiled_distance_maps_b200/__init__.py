@@ -63,6 +63,7 @@ _SIGS = {
     "tdm_box_muller": (_i32, [_vp, _vp, _i64, _vp, _vp]),
     "tdm_seam_discrepancy_noalloc": (_i32, [_vp, _P(CTiling), _vp, _vp]),
     "tdm_kabsch_stitch": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp, _vp]),
+    "tdm_refine_smacof": (_i32, [_vp, _vp, _i64, _vp, _i32, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -325,6 +326,18 @@ def seam_discrepancy_finalize(sums, tiling: Tiling, out, ctx: Context | None = N
     ctx.check(_lib.tdm_seam_discrepancy_finalize(ctx.handle, _ptr(sums, "sums", ctx), ctypes.byref(ct),
                                                  _ptr(out, "out", ctx), _stream(ctx)))
     return out
+
+
+def refine_smacof(maps, n_maps: int, coords, iterations: int, stress_out=None, ctx: Context | None = None):
+    """SMACOF refinement of ``coords`` ``[n][64][3]`` (in place) against
+    ``maps`` ``[n][64][64]`` (see tdm_refine_smacof)."""
+    ctx = ctx or context(maps.device.index)
+    _need(maps, n_maps * 4096, "maps")
+    _need(coords, n_maps * 192, "coords")
+    _need(stress_out, n_maps, "stress_out")
+    ctx.check(_lib.tdm_refine_smacof(ctx.handle, _ptr(maps, "maps", ctx), int(n_maps), _ptr(coords, "coords", ctx),
+                                     int(iterations), _ptr(stress_out, "stress_out", ctx), _stream(ctx)))
+    return coords
 
 
 def kabsch_stitch(coords, tiling: Tiling, chain_out, residual_out=None, ctx: Context | None = None):

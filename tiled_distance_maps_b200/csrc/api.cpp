@@ -371,6 +371,23 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "ddim_run launch");
 }
 
+// ---- refinement ---------------------------------------------------------------------
+
+tdm_status tdm_refine_smacof(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, int32_t iterations,
+                             float *stress_out, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (n_maps < 0) return fail(ctx, TDM_EINVAL, "n_maps < 0");
+    if (iterations < 0) return fail(ctx, TDM_EINVAL, "iterations < 0");
+    if (n_maps == 0) return TDM_OK;
+    tdm_status s;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, coords, "coords")) != TDM_OK) return s;
+    if (stress_out != nullptr && (reinterpret_cast<uintptr_t>(stress_out) & 3u))
+        return fail(ctx, TDM_EINVAL, "stress_out is not 4-byte aligned");
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_refine(maps, n_maps, coords, iterations, stress_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "refine launch");
+}
+
 // ---- stitching -----------------------------------------------------------------------
 
 tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling *tiling, float *chain_out,
