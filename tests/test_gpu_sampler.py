@@ -233,3 +233,27 @@ def test_invalid_arguments_are_rejected(tdm):
     # empty batches are a no-op
     tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.3, 0, tdm.Tiling(C=0, T=2, B=1))
     tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.3, 0, tdm.Tiling(C=1, T=2, B=0))
+
+
+def test_ddpm_ancestral_sampler_1000_steps(tdm):
+    # DDIM at eta = 1 with every training timestep is the DDPM ancestral
+    # sampler (posterior variance beta-tilde) used by the synchronisation
+    # experiments: the fused run against an oracle loop of DDPM steps
+    from oracle.ddim import ddpm_ancestral_step, eps_standin as oe, init_noise as oi
+    from oracle.seam import seam_project
+    T, B, S = 3, 2, 1000
+    t = tdm.Tiling(C=1, T=T, B=B, overlap=12, sync_every=1)
+    sch = tdm.Schedule(S, eta=1.0)
+    x0 = synth.chain_x0(17, 1, T)
+    maps = _maps(t)
+    tdm.ddim_run(sch, maps, dev(x0), 1.0, 0.1, 0.3, 23, t)
+    o = osched.Schedule(S=S, eta=1.0)
+    g = sample_ids(1, T, np.arange(B), B)
+    x = oi(23, g)
+    x0b = x0[:, :, None].astype(np.float64)
+    for tt in reversed(range(S)):
+        ec = oe(x, x0b, o.ab[tt], 0.1, stream_noise(23, philox.TAG_EPS_C, tt, g))
+        eu = oe(x, x0b, o.ab[tt], 0.3, stream_noise(23, philox.TAG_EPS_U, tt, g))
+        x = ddpm_ancestral_step(x, 2.0 * ec - eu, tt, o.betas, o.ab, stream_noise(23, philox.TAG_ETA, tt, g))
+        x = seam_project(x)
+    assert_maps_close(_as5(maps, t), x, TOL_MAP, "DDPM run")
