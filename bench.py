@@ -50,6 +50,11 @@ UNIT = "map-steps/s"
 OPS_PHILOX = 40
 OPS_BOX_MULLER_PAIR = 15
 QUADS_PER_MAP = 544
+# SMACOF refinement, per ordered bead pair and Guttman transform: 3 coordinate
+# differences, 3 for the squared distance, 1 reciprocal square root, 1 product
+# with D_ij, 3 accumulating FMAs
+OPS_GUTTMAN_PAIR = 11
+REFINE_ITERATIONS = 20    # stress within 2e-4 of its 100-iteration value from the MDS start
 
 
 def ops_per_map_step(n_streams: int) -> int:
@@ -320,6 +325,31 @@ def run_ours(args, rank, world, local_rank):
     step_ms = float(np.median([ps_ev[2 * i].elapsed_time(ps_ev[2 * i + 1]) for i in range(n_ps)]))
     del ec, eu
 
+    # the next rows beyond the step, each timed on its own over the step's output:
+    # SMACOF refinement of the 32,000 recovered coordinate sets and Kabsch
+    # stitching of the 32 tiles of each of the 1000 samples into one chain
+    L = 64 + (T - 1) * (64 - wl.overlap)
+    chains = torch.empty(B * L * 3, device=dev)
+    resid = torch.empty(B * (T - 1), device=dev)
+    stress = torch.empty(n_maps, device=dev)
+    coords0 = coords.clone()
+    nx = {}
+    for name, fn in (("kabsch_stitch", lambda: tdm.kabsch_stitch(coords0, tiling, chains, resid, ctx=ctx)),
+                     ("refine_smacof", lambda: tdm.refine_smacof(maps, n_maps, coords, REFINE_ITERATIONS, stress,
+                                                                 ctx=ctx))):
+        for _ in range(3):
+            fn()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * 10)]
+        for i in range(10):
+            coords.copy_(coords0)
+            ev[2 * i].record(stream)
+            fn()
+            ev[2 * i + 1].record(stream)
+        torch.cuda.synchronize()
+        nx[name] = float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(10)]))
+    flags |= tdm.ctx_sync(ctx)
+    del coords0, chains, resid, stress
+
     t = torch.tensor([ms, e2e_ms, float(np.mean(run_ms))], device=dev, dtype=torch.float64)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -357,6 +387,7 @@ def run_ours(args, rank, world, local_rank):
                               "frac": n_maps * 4 * 4096 * 4 / (step_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
                               "note": "one DDIM step of 32,000 maps, CFG w=1: read x, eps_c, eps_u, write x "
                                       "(64 KiB per map); timed separately from the step above"},
+            "next_rows": _next_rows(nx, n_maps, B, T, L, peak, float(peaks["hbm_gbs"])),
             "mds_not_converged": bool(flags & tdm.FLAG_MDS_NOT_CONVERGED),
             "peaks": kind,
         }
@@ -374,6 +405,26 @@ def run_ours(args, rank, world, local_rank):
                                               "float64 numpy"}
         print(json.dumps(line), flush=True)
     return 0
+
+
+def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
+    """Roofline lines of the kernels beyond the step (rank 0, this GPU)."""
+    ops = n_maps * REFINE_ITERATIONS * 64 * 64 * OPS_GUTTMAN_PAIR
+    st_bytes = n_maps * 192 * 4 + B * L * 3 * 4 + B * (T - 1) * 4
+    return {
+        "refine_smacof": {"kernel": "refine_kernel", "bound": "alu", "iterations": REFINE_ITERATIONS,
+                          "ms_per_launch": nx["refine_smacof"], "ops_per_launch": ops,
+                          "achieved": ops / (nx["refine_smacof"] / 1e3) / 1e12, "peak": alu_peak / 1e12,
+                          "unit": "Tops/s", "frac": ops / (nx["refine_smacof"] / 1e3) / alu_peak,
+                          "note": f"{n_maps} coordinate sets x {REFINE_ITERATIONS} Guttman transforms, "
+                                  f"{OPS_GUTTMAN_PAIR} lane-ops per ordered pair, plus the final stress"},
+        "kabsch_stitch": {"kernel": "stitch_kernel", "bound": "hbm", "ms_per_launch": nx["kabsch_stitch"],
+                          "bytes_per_launch": st_bytes,
+                          "achieved": st_bytes / (nx["kabsch_stitch"] / 1e3) / 1e9, "peak": hbm_gbs,
+                          "unit": "GB/s", "frac": st_bytes / (nx["kabsch_stitch"] / 1e3) / 1e9 / hbm_gbs,
+                          "note": f"{B} chains of {T} tiles: tile coordinates read, {L}-bead chains and "
+                                  "per-seam residuals written"},
+    }
 
 
 def _seam_chunks(n_seams, B):
