@@ -257,6 +257,20 @@ tdm_status tdm_seam_overlap_sums(tdm_ctx *ctx, const float *maps, const tdm_tili
 tdm_status tdm_seam_discrepancy_finalize(tdm_ctx *ctx, const float *sums, const tdm_tiling *tiling,
                                          float *out, tdm_stream stream);
 
+/* ---- non-overlap drift (ParaChromo §5.7, Table 8) ---------------------------
+ * How far the synchronised maps moved, outside the overlap blocks, from an
+ * independent run of the same seeds.  maps (synchronised) and ref
+ * (independent): device [C][T][B][64][64], read only, may alias.  The overlap
+ * blocks of tile k are its upper-left o x o block when k > 0 and its
+ * lower-right o x o block when k < T-1; all other entries count.
+ * tile_sums_out: device [C][T][2] = (sum |maps - ref|, sum |ref|) over the
+ * tile's B samples and counted entries.  drift_out (device [C], may be NULL):
+ * per chain, sum over its tiles of the first sum / sum of the second (NaN
+ * when both are 0, +inf when only the second is).  Sums of several shards of
+ * the samples add up.  tiling->sync_every is not used. */
+tdm_status tdm_nonoverlap_drift(tdm_ctx *ctx, const float *maps, const float *ref, const tdm_tiling *tiling,
+                                float *tile_sums_out, float *drift_out, tdm_stream stream);
+
 /* ---- the same without allocation -------------------------------------------
  * No counterpart in the paper: this entry point exists for callers that cannot
  * call cudaMalloc -- an application whose device memory is all handed to its

@@ -35,14 +35,14 @@ def nonoverlap_mask(T: int, k: int, overlap: int = 12, n: int = 64) -> np.ndarra
 def drift_sums(S: np.ndarray, V: np.ndarray, overlap: int = 12) -> np.ndarray:
     """``S, V [C][T][B][64][64]`` -> ``[C][T][2]`` = (sum |S - V|, sum |V|)
     over the samples and the non-overlap entries of each tile."""
-    S = np.asarray(S, dtype=np.float64)
-    V = np.asarray(V, dtype=np.float64)
     C, T = S.shape[:2]
     out = np.zeros((C, T, 2))
     for k in range(T):
         m = nonoverlap_mask(T, k, overlap, S.shape[-1])
-        out[:, k, 0] = np.abs(S[:, k] - V[:, k])[..., m].sum(axis=(1, 2))
-        out[:, k, 1] = np.abs(V[:, k])[..., m].sum(axis=(1, 2))
+        Sk = np.asarray(S[:, k], dtype=np.float64)
+        Vk = np.asarray(V[:, k], dtype=np.float64)
+        out[:, k, 0] = np.abs(Sk - Vk)[..., m].sum(axis=(1, 2))
+        out[:, k, 1] = np.abs(Vk)[..., m].sum(axis=(1, 2))
     return out
 
 

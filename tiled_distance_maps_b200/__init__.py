@@ -64,6 +64,7 @@ _SIGS = {
     "tdm_seam_discrepancy_noalloc": (_i32, [_vp, _P(CTiling), _vp, _vp]),
     "tdm_kabsch_stitch": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp, _vp]),
     "tdm_refine_smacof": (_i32, [_vp, _vp, _i64, _vp, _i32, _vp, _vp]),
+    "tdm_nonoverlap_drift": (_i32, [_vp, _vp, _vp, _P(CTiling), _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -338,6 +339,22 @@ def refine_smacof(maps, n_maps: int, coords, iterations: int, stress_out=None, c
     ctx.check(_lib.tdm_refine_smacof(ctx.handle, _ptr(maps, "maps", ctx), int(n_maps), _ptr(coords, "coords", ctx),
                                      int(iterations), _ptr(stress_out, "stress_out", ctx), _stream(ctx)))
     return coords
+
+
+def nonoverlap_drift(maps, ref, tiling: Tiling, tile_sums_out, drift_out=None, ctx: Context | None = None):
+    """Drift of ``maps`` from ``ref`` outside the overlap blocks: per-tile
+    sums ``[C][T][2]`` and optionally the per-chain ratio ``[C]`` (see
+    tdm_nonoverlap_drift)."""
+    ctx = ctx or context(maps.device.index)
+    _need(maps, tiling.n_maps * 4096, "maps")
+    _need(ref, tiling.n_maps * 4096, "ref")
+    _need(tile_sums_out, tiling.C * tiling.T * 2, "tile_sums_out")
+    _need(drift_out, tiling.C, "drift_out")
+    ct = tiling.c()
+    ctx.check(_lib.tdm_nonoverlap_drift(ctx.handle, _ptr(maps, "maps", ctx), _ptr(ref, "ref", ctx), ctypes.byref(ct),
+                                        _ptr(tile_sums_out, "tile_sums_out", ctx), _ptr(drift_out, "drift_out", ctx),
+                                        _stream(ctx)))
+    return tile_sums_out
 
 
 def kabsch_stitch(coords, tiling: Tiling, chain_out, residual_out=None, ctx: Context | None = None):

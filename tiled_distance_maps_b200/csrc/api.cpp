@@ -533,4 +533,25 @@ tdm_status tdm_seam_discrepancy(tdm_ctx *ctx, const float *maps, const tdm_tilin
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "seam discrepancy launch");
 }
 
+tdm_status tdm_nonoverlap_drift(tdm_ctx *ctx, const float *maps, const float *ref, const tdm_tiling *tiling,
+                                float *tile_sums_out, float *drift_out, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    Tiling t;
+    tdm_status s = check_tiling(ctx, tiling, &t);
+    if (s != TDM_OK) return s;
+    if (t.n_maps() == 0) return TDM_OK;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, ref, "ref")) != TDM_OK ||
+        (s = check_maps(ctx, tile_sums_out, "tile_sums_out")) != TDM_OK)
+        return s;
+    if (drift_out != nullptr && (reinterpret_cast<uintptr_t>(drift_out) & 3u))
+        return fail(ctx, TDM_EINVAL, "drift_out is not 4-byte aligned");
+    DeviceScope ds(ctx->device);
+    const int64_t tiles = (int64_t)t.C * t.T;
+    int chunks = tdm::drift_chunks(tiles, t.B);
+    if (chunks > 1 && (size_t)tiles * chunks * 2 > ctx->scratch_floats) chunks = 1;
+    cudaError_t e = tdm::launch_drift(maps, ref, t, ctx->d_scratch, chunks, tile_sums_out, drift_out,
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "drift launch");
+}
+
 }  // extern "C"
