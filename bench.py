@@ -16,6 +16,7 @@ line.  ``--impl reference`` times the float64 CPU oracle on a bounded sample.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import subprocess
@@ -55,6 +56,7 @@ QUADS_PER_MAP = 544
 # with D_ij, 3 accumulating FMAs
 OPS_GUTTMAN_PAIR = 11
 REFINE_ITERATIONS = 20    # stress within 2e-4 of its 100-iteration value from the MDS start
+SYNC_SWEEP = (0, 1, 2, 5, 10, 25, 50, 3, 7)    # 0 first: the independent run
 
 
 def ops_per_map_step(n_streams: int) -> int:
@@ -350,6 +352,48 @@ def run_ours(args, rank, world, local_rank):
     flags |= tdm.ctx_sync(ctx)
     del coords0, chains, resid, stress
 
+    # synchronisation-interval sweep (the wall ratio of synchronised to
+    # independent sampling, the non-overlap drift and the overlap discrepancy
+    # of each interval), and the drift kernel against its HBM roofline
+    ref_maps = torch.empty_like(maps)
+    tile_sums = torch.empty(T * 2, device=dev)
+    drift_ratio = torch.empty(1, device=dev)
+    sweep = {"K": [], "ms_per_run": [], "wall_ratio": [], "drift": [], "seam_discrepancy_mean": []}
+    ms_free = None
+    for K in SYNC_SWEEP:
+        tk = dataclasses.replace(tiling, sync_every=K)
+        out = ref_maps if K == 0 else maps
+        for _ in range(2):
+            tdm.ddim_run(sched, out, x0, wl.w, wl.s_c, wl.s_u, wl.seed, tk, ctx=ctx)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        for i in range(5):
+            ev[2 * i].record(stream)
+            tdm.ddim_run(sched, out, x0, wl.w, wl.s_c, wl.s_u, wl.seed, tk, ctx=ctx)
+            ev[2 * i + 1].record(stream)
+        torch.cuda.synchronize()
+        t_run = float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(5)]))
+        if K == 0:
+            ms_free = t_run
+            continue
+        sharded_seam_discrepancy(maps, tiling, sums, disc, ctx=ctx)
+        tdm.nonoverlap_drift(maps, ref_maps, tiling, tile_sums, drift_ratio, ctx=ctx)
+        sweep["K"].append(K)
+        sweep["ms_per_run"].append(t_run)
+        sweep["wall_ratio"].append(t_run / ms_free)
+        sweep["drift"].append(float(drift_ratio.item()))
+        sweep["seam_discrepancy_mean"].append(float(disc.mean().item()))
+    sweep["ms_unsynchronised"] = ms_free
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
+    for i in range(10):
+        ev[2 * i].record(stream)
+        tdm.nonoverlap_drift(maps, ref_maps, tiling, tile_sums, drift_ratio, ctx=ctx)
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize()
+    nx["nonoverlap_drift"] = float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(10)]))
+    nx["sync_sweep"] = sweep
+    flags |= tdm.ctx_sync(ctx)
+    del ref_maps
+
     t = torch.tensor([ms, e2e_ms, float(np.mean(run_ms))], device=dev, dtype=torch.float64)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -418,6 +462,16 @@ def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
                           "unit": "Tops/s", "frac": ops / (nx["refine_smacof"] / 1e3) / alu_peak,
                           "note": f"{n_maps} coordinate sets x {REFINE_ITERATIONS} Guttman transforms, "
                                   f"{OPS_GUTTMAN_PAIR} lane-ops per ordered pair, plus the final stress"},
+        "nonoverlap_drift": {"kernel": "drift_sums_kernel", "bound": "hbm", "ms_per_launch": nx["nonoverlap_drift"],
+                             "bytes_per_launch": 2 * n_maps * 4096 * 4,
+                             "achieved": 2 * n_maps * 4096 * 4 / (nx["nonoverlap_drift"] / 1e3) / 1e9,
+                             "peak": hbm_gbs, "unit": "GB/s",
+                             "frac": 2 * n_maps * 4096 * 4 / (nx["nonoverlap_drift"] / 1e3) / 1e9 / hbm_gbs,
+                             "note": "synchronised and independent maps read once (32 KiB per map pair)"},
+        "sync_interval_sweep": dict(nx["sync_sweep"], note=(
+            "the fused run with the projection every K steps against the same run without it (K = 0); "
+            "drift: non-overlap drift from that run; the ideal-denoiser stand-in acts entry by entry, "
+            "so it is 0, and the discrepancy is 0 whenever K divides S")),
         "kabsch_stitch": {"kernel": "stitch_kernel", "bound": "hbm", "ms_per_launch": nx["kabsch_stitch"],
                           "bytes_per_launch": st_bytes,
                           "achieved": st_bytes / (nx["kabsch_stitch"] / 1e3) / 1e9, "peak": hbm_gbs,
