@@ -90,7 +90,10 @@ typedef struct tdm_tiling {
 
 /* Creates a context on CUDA device `device` (allocates its status word and
  * scratch).  *out receives the handle.  Errors: TDM_EINVAL (out NULL or bad
- * device), TDM_ENOMEM, TDM_ECUDA. */
+ * device), TDM_ENOMEM, TDM_ECUDA.  The calls that keep intermediate results
+ * in the scratch (tdm_seam_discrepancy, tdm_nonoverlap_drift,
+ * tdm_kabsch_stitch) must not overlap on the GPU for one context: issue them
+ * on one stream, or give each stream its own context. */
 tdm_status tdm_ctx_create(tdm_ctx **out, int32_t device);
 
 /* Frees everything the context owns.  NULL is ignored. */
@@ -205,7 +208,9 @@ tdm_status tdm_refine_smacof(tdm_ctx *ctx, const float *maps, int64_t n_maps, fl
  * frame.  chain_out: device [C][B][L][3], L = 64 + (T-1)(64-o); an overlap
  * bead is the mean of its two aligned copies.  residual_out: device
  * [C][B][T-1] (may be NULL), the RMSD over the o beads of each seam after the
- * alignment, in the coordinates' units.  Needs overlap >= 3 when T > 1. */
+ * alignment, in the coordinates' units.  Needs overlap >= 3 when T > 1.
+ * The tiles' maps go through context scratch in chunks of (chain, sample)
+ * pairs. */
 tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling *tiling, float *chain_out,
                              float *residual_out, tdm_stream stream);
 
@@ -267,7 +272,8 @@ tdm_status tdm_seam_discrepancy_finalize(tdm_ctx *ctx, const float *sums, const 
  * tile's B samples and counted entries.  drift_out (device [C], may be NULL):
  * per chain, sum over its tiles of the first sum / sum of the second (NaN
  * when both are 0, +inf when only the second is).  Sums of several shards of
- * the samples add up.  tiling->sync_every is not used. */
+ * the samples add up.  tiling->sync_every is not used.  When there are few
+ * tiles, partial sums over chunks of samples go through context scratch. */
 tdm_status tdm_nonoverlap_drift(tdm_ctx *ctx, const float *maps, const float *ref, const tdm_tiling *tiling,
                                 float *tile_sums_out, float *drift_out, tdm_stream stream);
 

@@ -33,7 +33,8 @@ def _run(tdm, X, T, overlap):
 
 
 @pytest.mark.parametrize("C,T,B,o,noise", [(2, 5, 3, 12, 0.05), (1, 32, 8, 12, 0.02), (2, 40, 3, 8, 0.05),
-                                           (1, 3, 2, 32, 0.0), (3, 1, 2, 12, 0.0)])
+                                           (1, 3, 2, 32, 0.0), (3, 1, 2, 12, 0.0), (2, 6, 3, 7, 0.05),
+                                           (1, 4, 5, 5, 0.0)])
 def test_stitch_matches_oracle(tdm, C, T, B, o, noise):
     X, _, _ = synth.tile_coords(T * 7 + B, C, T, B, overlap=o, noise=noise)
     got, res = _run(tdm, X, T, o)
@@ -62,3 +63,39 @@ def test_stitch_chromosome_chain_full_size(tdm):
     scale = np.abs(ref).max(axis=(-1, -2))
     assert (np.abs(got[:, idx] - ref).max(axis=(-1, -2)) / scale).max() <= TOL_CHAIN
     assert (np.abs(res[:, idx] - rref) / np.maximum(rref, 2e-5)).max() <= TOL_RESID
+
+
+def test_stitch_pairs_over_several_scratch_chunks(tdm):
+    # 4000 samples of a 32-tile chain: more (chain, sample) pairs than one
+    # chunk of tile maps in the context scratch holds; chains on both sides of
+    # a chunk boundary through the oracle
+    C, T, B = 1, 32, 4000
+    X, _, _ = synth.tile_coords(7, C, T, B, noise=0.02)
+    got, res = _run(tdm, X, T, 12)
+    idx = np.array([0, 1, 3155, 3156, 3157, 3158, 3999])
+    ref, rref = ostitch.stitch(X[:, :, idx].astype(np.float64))
+    scale = np.abs(ref).max(axis=(-1, -2))
+    assert (np.abs(got[:, idx] - ref).max(axis=(-1, -2)) / scale).max() <= TOL_CHAIN
+    assert (np.abs(res[:, idx] - rref) / np.maximum(rref, 2e-5)).max() <= TOL_RESID
+
+
+def test_stitch_longest_chains(tdm):
+    # two samples of a chain of 65,535 tiles (the most a chain may have): the
+    # tile maps of one pair fill most of the context scratch, so each pair is a
+    # chunk of its own.  float32 composition over 65,534 seams drifts, so the
+    # oracle checks the first 40 tiles and sampled seams, and every bond of
+    # both chains is checked against the walk
+    C, T, B, o = 1, 65535, 2, 12
+    X, walks, _ = synth.tile_coords(3, C, T, B, noise=0.0)
+    got, res = _run(tdm, X, T, o)
+    assert np.isfinite(got).all()
+    L40 = 64 + 39 * 52
+    ref, _ = ostitch.stitch(X[:, :40].astype(np.float64), o)
+    for b in range(B):
+        assert np.abs(got[0, b, :L40] - ref[0, b]).max() / np.abs(ref[0, b]).max() <= TOL_CHAIN
+        for k in np.random.default_rng(b).choice(T - 1, 30, replace=False):
+            _, _, r = ostitch.procrustes(X[0, k, b, 52:].astype(np.float64), X[0, k + 1, b, :o].astype(np.float64))
+            assert abs(res[0, b, k] - r) <= 2e-5 * float(np.abs(X[0, k, b]).max())
+        bond = np.linalg.norm(np.diff(got[0, b], axis=0), axis=1)
+        walk_bond = np.linalg.norm(np.diff(walks[0, b], axis=0), axis=1)
+        assert np.abs(bond - walk_bond).max() <= 0.05

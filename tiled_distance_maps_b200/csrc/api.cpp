@@ -403,8 +403,8 @@ tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling
     if (residual_out != nullptr && (reinterpret_cast<uintptr_t>(residual_out) & 3u))
         return fail(ctx, TDM_EINVAL, "residual_out is not 4-byte aligned");
     DeviceScope ds(ctx->device);
-    cudaError_t e = tdm::launch_stitch(coords, t, chain_out, t.T > 1 ? residual_out : nullptr,
-                                       static_cast<cudaStream_t>(stream));
+    cudaError_t e = tdm::launch_stitch(coords, t, chain_out, t.T > 1 ? residual_out : nullptr, ctx->d_scratch,
+                                       ctx->scratch_floats, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "stitch launch");
 }
 

@@ -79,7 +79,8 @@ cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigva
 cudaError_t launch_pdist(const float *coords, int64_t n, float *maps, cudaStream_t st);
 cudaError_t launch_refine(const float *maps, int64_t n, float *coords, int iterations, float *stress,
                           cudaStream_t st);
-cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, cudaStream_t st);
+cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, float *scratch,
+                          size_t scratch_floats, cudaStream_t st);
 cudaError_t launch_philox(const uint32_t *ctr, int64_t n, uint64_t seed, uint32_t *out, cudaStream_t st);
 cudaError_t launch_box_muller(const uint32_t *words, int64_t n_pairs, float *z, cudaStream_t st);
 

@@ -9,8 +9,9 @@
 // maps compose along the chain into tile 0's frame; overlap beads take the
 // mean of their two aligned copies.
 //
-// One warp per (chain, sample); lane k handles seam k and tile k of a chunk
-// of 32 tiles, and a shuffle scan composes the maps.
+// Two passes over chunks of (chain, sample) pairs whose tile maps fit the
+// context scratch: one warp per pair aligns the seams and composes the maps by
+// a shuffle scan, 32 tiles at a time; then one thread per chain bead places it.
 #include "common.cuh"
 
 namespace tdm {
@@ -216,62 +217,150 @@ __device__ Rigid align_seam(const float *P, const float *Q, int o, float *rmsd) 
     return g;
 }
 
-__global__ void __launch_bounds__(128) stitch_kernel(const float *__restrict__ coords, int C, int T, int B, int o,
-                                                     float *__restrict__ chain, float *__restrict__ resid) {
+
+// Seam maps of one chunk of 32 tiles, composed into tile 0's frame (warp-wide;
+// lane l ends with G_{k0+l}); P / Q: lane l's seam k0+l beads (tile k0+l's
+// last o, tile k0+l+1's first o), read only when that seam exists.  carry /
+// carry_prev hold G_{k0} / G_{k0-1} on entry and G_{k0+32} / G_{k0+31} on
+// return.  Residuals of the chunk's seams are written when resid is not NULL.
+__device__ __forceinline__ Rigid chunk_maps(const float *P, const float *Q, int T, int o, int k0, int64_t pair,
+                                            float *__restrict__ resid, Rigid &carry, Rigid &carry_prev) {
     const int lane = threadIdx.x & 31;
-    const int64_t nw = (int64_t)C * B;
+    const int k = k0 + lane;
+    Rigid tk = identity();    // seam k: tile k+1 onto tile k
+    if (k < T - 1) {
+        float r;
+        tk = align_seam(P, Q, o, &r);
+        if (resid != nullptr) resid[pair * (T - 1) + k] = r;
+    }
+    Rigid sk = tk;    // inclusive scan: t_{k0} o ... o t_k
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const Rigid prev = shfl_up(sk, d);
+        if (lane >= d) sk = compose(prev, sk);
+    }
+    const Rigid gnext = compose(carry, sk);    // G_{k+1}
+    Rigid gk = shfl_up(gnext, 1);               // G_k
+    if (lane == 0) gk = carry;
+    carry_prev = shfl_idx(gk, 31);
+    carry = shfl_idx(gnext, 31);
+    return gk;
+}
+
+// 4-byte asynchronous global -> shared copy (the copies of a chunk are all in
+// flight before the warp waits for them)
+__device__ __forceinline__ void async_copy4(float *dst, const float *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+
+// Pass 1: one warp (one CTA) per (chain, sample) of pairs [pair0, pair0 + n):
+// the seam beads of 32 tiles at a time staged in shared memory by coalesced
+// warp-wide asynchronous copies (per-lane stride 3o+1 floats, odd, so the lanes' reads do
+// not conflict), then every tile's map into gmaps[(pair - pair0) * T + k] and
+// the residuals into resid.
+__global__ void __launch_bounds__(32) stitch_align_kernel(const float *__restrict__ coords, int T, int B, int o,
+                                                          int64_t pair0, Rigid *__restrict__ gmaps,
+                                                          float *__restrict__ resid) {
+    extern __shared__ float sbeads[];    // [2][32][3o+1]: P then Q per lane
+    const int lane = threadIdx.x;
+    const int64_t q = blockIdx.x;
+    const int64_t pair = pair0 + q;
+    const int c = (int)(pair / B), b = (int)(pair - (int64_t)(pair / B) * B);
     const int s = kN - o;
-    const int64_t L = kN + (int64_t)(T - 1) * s;
-    for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < nw;
-         w += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-        const int c = (int)(w / B), b = (int)(w - (int64_t)c * B);
-        float *out = chain + w * L * 3;
-        Rigid carry = identity();        // G_k0: tile k0 into tile 0's frame
-        Rigid carry_prev = identity();   // G_{k0-1}
-        for (int k0 = 0; k0 < T; k0 += 32) {
-            const int k = k0 + lane;
-            // seam k: tile k+1 onto tile k
-            Rigid tk = identity();
-            if (k < T - 1) {
-                const float *Pk = coords + (((int64_t)c * T + k) * B + b) * (kN * 3) + s * 3;
-                const float *Qk = coords + (((int64_t)c * T + k + 1) * B + b) * (kN * 3);
-                float r;
-                tk = align_seam(Pk, Qk, o, &r);
-                if (resid != nullptr) resid[w * (T - 1) + k] = r;
+    const int n3 = 3 * o, ld = 3 * o + 1;
+    float *sP = sbeads, *sQ = sbeads + 32 * ld;
+    Rigid carry = identity(), carry_prev = identity();
+    for (int k0 = 0; k0 < T; k0 += 32) {
+        const int nseam = min(32, T - 1 - k0);    // seams k0 .. k0+nseam-1
+        __syncwarp();
+        for (int r = 0; r < nseam; ++r) {
+            const float *Pg = coords + (((int64_t)c * T + k0 + r) * B + b) * (kN * 3) + s * 3;
+            const float *Qg = coords + (((int64_t)c * T + k0 + r + 1) * B + b) * (kN * 3);
+            for (int i = lane; i < n3; i += 32) {
+                async_copy4(sP + r * ld + i, Pg + i);
+                async_copy4(sQ + r * ld + i, Qg + i);
             }
-            // inclusive scan within the chunk: S_k = t_k0 o ... o t_k
-            Rigid sk = tk;
+        }
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        const Rigid gk = chunk_maps(sP + lane * ld, sQ + lane * ld, T, o, k0, pair, resid, carry, carry_prev);
+        if (k0 + lane < T) gmaps[q * T + k0 + lane] = gk;
+    }
+}
+
+__device__ __forceinline__ Rigid load_map(const Rigid *g) {
+    const float4 *v = reinterpret_cast<const float4 *>(g);
+    const float4 a = __ldg(v), b = __ldg(v + 1), c = __ldg(v + 2);
+    Rigid o;
+    o.r[0] = a.x, o.r[1] = a.y, o.r[2] = a.z, o.r[3] = a.w;
+    o.r[4] = b.x, o.r[5] = b.y, o.r[6] = b.z, o.r[7] = b.w;
+    o.r[8] = c.x, o.t[0] = c.y, o.t[1] = c.z, o.t[2] = c.w;
+    return o;
+}
+
+// Pass 2: one thread per G beads of the chains of pairs [pair0, pair0 + n).
+// Tile k owns chain positions [k s, k s + s), the last tile [k s, k s + 64);
+// the first o beads of tile k > 0 are the mean of tile k-1's and tile k's
+// aligned copies.  G = 4 needs o % 4 == 0: four beads then stay in one tile
+// and on one side of the overlap boundary, and their 12 coordinates are
+// 16-byte aligned in the tile and in the chain.  32-bit indices: a chunk holds
+// n L <= (scratch / 12T) * 64T beads, and pairs < 2^31 is checked by the caller.
+template <int G>
+__global__ void __launch_bounds__(256) stitch_place_kernel(const float *__restrict__ coords, int T, int B, int o,
+                                                           int pair0, int n, const Rigid *__restrict__ gmaps,
+                                                           float *__restrict__ chain) {
+    const int s = kN - o;
+    const int L = kN + (T - 1) * s;
+    const int LG = L / G;
+    const int total = n * LG;
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
+        const int q = idx / LG;
+        const int p = (idx - q * LG) * G;
+        const int pair = pair0 + q;
+        const int c = pair / B, b = pair - (pair / B) * B;
+        int k = p / s;
+        if (k > T - 1) k = T - 1;
+        const int j = p - k * s;
+        float x[3 * G], y[3 * G];
+        const float *xk = coords + (((int64_t)c * T + k) * B + b) * (kN * 3) + 3 * j;
+        if constexpr (G == 4) {
 #pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const Rigid prev = shfl_up(sk, d);
-                if (lane >= d) sk = compose(prev, sk);
-            }
-            const Rigid gnext = compose(carry, sk);          // G_{k+1}
-            Rigid gk = shfl_up(gnext, 1);                     // G_k
-            if (lane == 0) gk = carry;
-            Rigid gkm1 = shfl_up(gk, 1);                      // G_{k-1}
-            if (lane == 0) gkm1 = carry_prev;
-            if (k < T) {
-                const float *Xk = coords + (((int64_t)c * T + k) * B + b) * (kN * 3);
-                float *dst = out + (int64_t)k * s * 3;
-                // own beads: not the left overlap (written below, averaged) and
-                // not the right overlap (the next tile's lane averages it)
-                const int j0 = k == 0 ? 0 : o;
-                const int j1 = k == T - 1 ? kN : s;
-                for (int j = j0; j < j1; ++j) apply(gk, Xk + 3 * j, dst + 3 * j);
-                if (k > 0) {
-                    const float *Xp = coords + (((int64_t)c * T + k - 1) * B + b) * (kN * 3) + s * 3;
-                    for (int j = 0; j < o; ++j) {
-                        float y1[3], y2[3];
-                        apply(gkm1, Xp + 3 * j, y1);
-                        apply(gk, Xk + 3 * j, y2);
+            for (int v = 0; v < 3; ++v) *reinterpret_cast<float4 *>(x + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xk) + v);
+        } else {
 #pragma unroll
-                        for (int d = 0; d < 3; ++d) dst[3 * j + d] = 0.5f * (y1[d] + y2[d]);
-                    }
-                }
+            for (int v = 0; v < 3 * G; ++v) x[v] = __ldg(xk + v);
+        }
+        const Rigid gk = load_map(gmaps + (int64_t)q * T + k);
+#pragma unroll
+        for (int u = 0; u < G; ++u) apply(gk, x + 3 * u, y + 3 * u);
+        if (k > 0 && j < o) {
+            const float *xp = coords + (((int64_t)c * T + k - 1) * B + b) * (kN * 3) + 3 * (s + j);
+            if constexpr (G == 4) {
+#pragma unroll
+                for (int v = 0; v < 3; ++v)
+                    *reinterpret_cast<float4 *>(x + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xp) + v);
+            } else {
+#pragma unroll
+                for (int v = 0; v < 3 * G; ++v) x[v] = __ldg(xp + v);
             }
-            carry_prev = shfl_idx(gk, 31);
-            carry = shfl_idx(gnext, 31);
+            const Rigid gp = load_map(gmaps + (int64_t)q * T + k - 1);
+#pragma unroll
+            for (int u = 0; u < G; ++u) {
+                float y1[3];
+                apply(gp, x + 3 * u, y1);
+#pragma unroll
+                for (int d = 0; d < 3; ++d) y[3 * u + d] = 0.5f * (y1[d] + y[3 * u + d]);
+            }
+        }
+        float *dst = chain + ((int64_t)pair * L + p) * 3;
+        if constexpr (G == 4) {
+#pragma unroll
+            for (int v = 0; v < 3; ++v) reinterpret_cast<float4 *>(dst)[v] = *reinterpret_cast<const float4 *>(y + 4 * v);
+        } else {
+#pragma unroll
+            for (int v = 0; v < 3 * G; ++v) dst[v] = y[v];
         }
     }
 }
@@ -281,16 +370,33 @@ __global__ void __launch_bounds__(128) stitch_kernel(const float *__restrict__ c
 
 namespace tdm {
 
-cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, cudaStream_t st) {
-    const int64_t warps = (int64_t)t.C * t.B;
-    if (warps <= 0) return cudaSuccess;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t grid = (warps + 3) / 4;
-    if (grid > (int64_t)sms * 16) grid = (int64_t)sms * 16;
-    stitch_kernel<<<(int)grid, 128, 0, st>>>(coords, t.C, t.T, t.B, t.T > 1 ? t.overlap : 0, chain, resid);
-    return cudaGetLastError();
+cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, float *scratch,
+                          size_t scratch_floats, cudaStream_t st) {
+    const int64_t pairs = (int64_t)t.C * t.B;
+    if (pairs <= 0) return cudaSuccess;
+    if (pairs > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const int o = t.T > 1 ? t.overlap : 0;
+    const int64_t per_pair = (int64_t)t.T * (int64_t)(sizeof(Rigid) / sizeof(float));
+    // T <= 65535 (checked with the tiling) keeps one pair's maps within the scratch
+    const int64_t chunk = scratch == nullptr ? 0 : (int64_t)scratch_floats / per_pair;
+    if (chunk < 1) return cudaErrorInvalidValue;
+    Rigid *gmaps = reinterpret_cast<Rigid *>(scratch);
+    for (int64_t p0 = 0; p0 < pairs; p0 += chunk) {
+        const int64_t n = pairs - p0 < chunk ? pairs - p0 : chunk;
+        const size_t smem = sizeof(float) * 2 * 32 * (3 * o + 1);
+        stitch_align_kernel<<<(unsigned)n, 32, smem, st>>>(coords, t.T, t.B, o, p0, gmaps, resid);
+        const int64_t beads = n * (kN + (int64_t)(t.T - 1) * (kN - o));
+        const bool vec = o % 4 == 0;
+        int64_t blocks = ((vec ? beads / 4 : beads) + 255) / 256;
+        if (blocks > 148LL * 64) blocks = 148LL * 64;
+        if (vec)
+            stitch_place_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(coords, t.T, t.B, o, (int)p0, (int)n, gmaps, chain);
+        else
+            stitch_place_kernel<1><<<(unsigned)blocks, 256, 0, st>>>(coords, t.T, t.B, o, (int)p0, (int)n, gmaps, chain);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace tdm
