@@ -335,20 +335,12 @@ def run_ours(args, rank, world, local_rank):
     resid = torch.empty(B * (T - 1), device=dev)
     stress = torch.empty(n_maps, device=dev)
     coords0 = coords.clone()
+    l2_flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)    # 256 MiB > 126 MB L2
     nx = {}
     for name, fn in (("kabsch_stitch", lambda: tdm.kabsch_stitch(coords0, tiling, chains, resid, ctx=ctx)),
                      ("refine_smacof", lambda: tdm.refine_smacof(maps, n_maps, coords, REFINE_ITERATIONS, stress,
                                                                  ctx=ctx))):
-        for _ in range(3):
-            fn()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * 10)]
-        for i in range(10):
-            coords.copy_(coords0)
-            ev[2 * i].record(stream)
-            fn()
-            ev[2 * i + 1].record(stream)
-        torch.cuda.synchronize()
-        nx[name] = float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(10)]))
+        nx[name] = _time_flushed(fn, stream, l2_flush)
     flags |= tdm.ctx_sync(ctx)
     del coords0, chains, resid, stress
 
@@ -383,13 +375,9 @@ def run_ours(args, rank, world, local_rank):
         sweep["drift"].append(float(drift_ratio.item()))
         sweep["seam_discrepancy_mean"].append(float(disc.mean().item()))
     sweep["ms_unsynchronised"] = ms_free
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(20)]
-    for i in range(10):
-        ev[2 * i].record(stream)
-        tdm.nonoverlap_drift(maps, ref_maps, tiling, tile_sums, drift_ratio, ctx=ctx)
-        ev[2 * i + 1].record(stream)
-    torch.cuda.synchronize()
-    nx["nonoverlap_drift"] = float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(10)]))
+    nx["nonoverlap_drift"] = _time_flushed(
+        lambda: tdm.nonoverlap_drift(maps, ref_maps, tiling, tile_sums, drift_ratio, ctx=ctx), stream, l2_flush)
+    del l2_flush
     nx["sync_sweep"] = sweep
     flags |= tdm.ctx_sync(ctx)
     del ref_maps
@@ -451,11 +439,31 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def _time_flushed(fn, stream, flush, n: int = 10) -> float:
+    """Median ms of ``n`` calls of ``fn``, each timed by its own events after a
+    write of ``flush`` (larger than L2) that also keeps the GPU busy while the
+    host enqueues the call; 3 untimed calls first.  Each call does the same
+    work whatever its inputs hold."""
+    import torch
+    for _ in range(3):
+        fn()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n)]
+    for i in range(n):
+        flush.zero_()
+        ev[2 * i].record(stream)
+        fn()
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize()
+    return float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n)]))
+
+
 def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
     """Roofline lines of the kernels beyond the step (rank 0, this GPU)."""
     ops = n_maps * REFINE_ITERATIONS * 64 * 64 * OPS_GUTTMAN_PAIR
     st_bytes = n_maps * 192 * 4 + B * L * 3 * 4 + B * (T - 1) * 4
     return {
+        "timing": "each call timed alone by CUDA events after a 256 MiB write that flushes L2 (median of 10); "
+                  "the sweep's runs back to back (their working set exceeds L2)",
         "refine_smacof": {"kernel": "refine_kernel", "bound": "alu", "iterations": REFINE_ITERATIONS,
                           "ms_per_launch": nx["refine_smacof"], "ops_per_launch": ops,
                           "achieved": ops / (nx["refine_smacof"] / 1e3) / 1e12, "peak": alu_peak / 1e12,

@@ -323,33 +323,39 @@ __global__ void __launch_bounds__(256) stitch_place_kernel(const float *__restri
         int k = p / s;
         if (k > T - 1) k = T - 1;
         const int j = p - k * s;
-        float x[3 * G], y[3 * G];
+        // both rounds of loads (the tile's beads and map; for overlap beads also
+        // the previous tile's) are issued before any arithmetic
+        const bool ov = k > 0 && j < o;
+        float x[3 * G], xp[3 * G], y[3 * G];
         const float *xk = coords + (((int64_t)c * T + k) * B + b) * (kN * 3) + 3 * j;
+        const float *xq = coords + (((int64_t)c * T + (ov ? k - 1 : k)) * B + b) * (kN * 3) + 3 * (s + j);
+        const Rigid gk = load_map(gmaps + (int64_t)q * T + k);
+        Rigid gp = gk;
         if constexpr (G == 4) {
 #pragma unroll
             for (int v = 0; v < 3; ++v) *reinterpret_cast<float4 *>(x + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xk) + v);
+            if (ov) {
+#pragma unroll
+                for (int v = 0; v < 3; ++v)
+                    *reinterpret_cast<float4 *>(xp + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xq) + v);
+                gp = load_map(gmaps + (int64_t)q * T + k - 1);
+            }
         } else {
 #pragma unroll
             for (int v = 0; v < 3 * G; ++v) x[v] = __ldg(xk + v);
+            if (ov) {
+#pragma unroll
+                for (int v = 0; v < 3 * G; ++v) xp[v] = __ldg(xq + v);
+                gp = load_map(gmaps + (int64_t)q * T + k - 1);
+            }
         }
-        const Rigid gk = load_map(gmaps + (int64_t)q * T + k);
 #pragma unroll
         for (int u = 0; u < G; ++u) apply(gk, x + 3 * u, y + 3 * u);
-        if (k > 0 && j < o) {
-            const float *xp = coords + (((int64_t)c * T + k - 1) * B + b) * (kN * 3) + 3 * (s + j);
-            if constexpr (G == 4) {
-#pragma unroll
-                for (int v = 0; v < 3; ++v)
-                    *reinterpret_cast<float4 *>(x + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xp) + v);
-            } else {
-#pragma unroll
-                for (int v = 0; v < 3 * G; ++v) x[v] = __ldg(xp + v);
-            }
-            const Rigid gp = load_map(gmaps + (int64_t)q * T + k - 1);
+        if (ov) {
 #pragma unroll
             for (int u = 0; u < G; ++u) {
                 float y1[3];
-                apply(gp, x + 3 * u, y1);
+                apply(gp, xp + 3 * u, y1);
 #pragma unroll
                 for (int d = 0; d < 3; ++d) y[3 * u + d] = 0.5f * (y1[d] + y[3 * u + d]);
             }
