@@ -69,8 +69,12 @@ def alu_peak_ops(sms: int = 148, clock_ghz: float = 1.965) -> float:
     return sms * 128 * clock_ghz * 1e9
 
 
-RUN_SOURCES = ["tiled_distance_maps_b200/csrc/sampler.cu", "tiled_distance_maps_b200/csrc/common.cuh",
-               "tiled_distance_maps_b200/csrc/internal.h"]
+# the files that hold each kernel's device code (a change to them voids the
+# DRAM traffic recorded by an earlier ncu capture)
+RUN_SOURCES = ["tiled_distance_maps_b200/csrc/sampler.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
+REFINE_SOURCES = ["tiled_distance_maps_b200/csrc/refine.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
+DRIFT_SOURCES = ["tiled_distance_maps_b200/csrc/drift.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
+STITCH_SOURCES = ["tiled_distance_maps_b200/csrc/stitch.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
 
 
 def profiled_traffic(summary: str, sources) -> int | None:
@@ -468,6 +472,7 @@ def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
                           "ms_per_launch": nx["refine_smacof"], "ops_per_launch": ops,
                           "achieved": ops / (nx["refine_smacof"] / 1e3) / 1e12, "peak": alu_peak / 1e12,
                           "unit": "Tops/s", "frac": ops / (nx["refine_smacof"] / 1e3) / alu_peak,
+                          "traffic": profiled_traffic("refine_kernel_chain32_b1000_cfg.md", REFINE_SOURCES),
                           "note": f"{n_maps} coordinate sets x {REFINE_ITERATIONS} Guttman transforms, "
                                   f"{OPS_GUTTMAN_PAIR} lane-ops per ordered pair, plus the final stress"},
         "nonoverlap_drift": {"kernel": "drift_sums_kernel", "bound": "hbm", "ms_per_launch": nx["nonoverlap_drift"],
@@ -475,6 +480,7 @@ def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
                              "achieved": 2 * n_maps * 4096 * 4 / (nx["nonoverlap_drift"] / 1e3) / 1e9,
                              "peak": hbm_gbs, "unit": "GB/s",
                              "frac": 2 * n_maps * 4096 * 4 / (nx["nonoverlap_drift"] / 1e3) / 1e9 / hbm_gbs,
+                             "traffic": profiled_traffic("drift_sums_kernel_chain32_b1000_cfg.md", DRIFT_SOURCES),
                              "note": "synchronised and independent maps read once (32 KiB per map pair)"},
         "sync_interval_sweep": dict(nx["sync_sweep"], note=(
             "the fused run with the projection every K steps against the same run without it (K = 0); "
@@ -484,6 +490,7 @@ def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
                           "bytes_per_launch": st_bytes,
                           "achieved": st_bytes / (nx["kabsch_stitch"] / 1e3) / 1e9, "peak": hbm_gbs,
                           "unit": "GB/s", "frac": st_bytes / (nx["kabsch_stitch"] / 1e3) / 1e9 / hbm_gbs,
+                          "traffic": profiled_traffic("stitch_chain32_b1000_cfg.md", STITCH_SOURCES),
                           "note": f"{B} chains of {T} tiles: tile coordinates read, {L}-bead chains and "
                                   "per-seam residuals written"},
     }
