@@ -291,25 +291,46 @@ def run_ours(args, rank, world, local_rank):
     run_ms = [ev_run[2 * i].elapsed_time(ev_run[2 * i + 1]) for i in range(args.steps)]
     flags |= tdm.ctx_sync(ctx)
 
-    # end to end through the public API from host buffers
+    # end to end through the public API from host buffers: every step uploads
+    # x0 from pinned memory and reads back its coordinates, eigenvalues and
+    # Eq. (6).  The outputs are double-buffered and read back on a copy stream,
+    # so step i's read-back overlaps step i+1's kernels; the timed region ends
+    # after the last read-back.
     pinned_x0 = x0_host.pin_memory()
-    h_coords = torch.empty(n_maps * 192, dtype=torch.float32).pin_memory()
-    h_eig = torch.empty(n_maps * 3, dtype=torch.float32).pin_memory()
-    h_disc = torch.empty(T - 1, dtype=torch.float32).pin_memory()
+    dev_out = [(coords, eig, disc), (torch.empty_like(coords), torch.empty_like(eig), torch.empty_like(disc))]
+    host_out = [tuple(torch.empty(t.numel(), dtype=torch.float32).pin_memory() for t in bufs) for bufs in dev_out]
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def step_into(cb, eb, db):
+        tdm.ddim_run(sched, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, tiling, ctx=ctx)
+        tdm.mds_recover(maps, n_maps, cb, eb, ctx=ctx)
+        tdm.pairwise_dist(cb, n_maps, rec, ctx=ctx)
+        sharded_seam_discrepancy(rec, tiling, sums, db, ctx=ctx)
+
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e_start.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        j = i % 2
+        if i >= 2:
+            stream.wait_event(copied[j])          # buffer j's previous read-back is done
         x0.copy_(pinned_x0, non_blocking=True)
-        step()
-        h_coords.copy_(coords, non_blocking=True)
-        h_eig.copy_(eig, non_blocking=True)
-        h_disc.copy_(disc, non_blocking=True)
+        step_into(*dev_out[j])
+        ready = torch.cuda.Event()
+        ready.record(stream)
+        copy_stream.wait_event(ready)
+        with torch.cuda.stream(copy_stream):
+            for h, d in zip(host_out[j], dev_out[j]):
+                h.copy_(d, non_blocking=True)
+            copied[j].record(copy_stream)
+    stream.wait_stream(copy_stream)
     e_stop.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e_start.elapsed_time(e_stop)
+    del dev_out, host_out
 
     # the per-step path (the kernel a real model would drive: eps materialised
     # by the model, here by the stand-in), timed on its own after the step:
@@ -414,7 +435,10 @@ def run_ours(args, rank, world, local_rank):
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
             "e2e": {"value": map_steps * args.steps / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": x0_host.numel() * 4,
-                    "d2h_bytes_per_step": (n_maps * 195 + (T - 1)) * 4},
+                    "d2h_bytes_per_step": (n_maps * 195 + (T - 1)) * 4,
+                    "note": "x0 uploaded from pinned memory and coordinates, eigenvalues and Eq. (6) read back "
+                            "every step; outputs double-buffered, read-backs on a copy stream overlap the next "
+                            "step"},
             "gpu_launches": launches_per_step * args.steps,
             "per_step_path": {"kernel": "ddim_step_kernel", "bound": "hbm", "ms_per_launch": step_ms,
                               "bytes_per_launch": n_maps * 4 * 4096 * 4,
