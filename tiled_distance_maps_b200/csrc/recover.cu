@@ -345,26 +345,47 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
     }
 }
 
+// Distance reconstruction: kPdistMaps maps per CTA iteration, their
+// coordinates staged as structure of arrays (x[64], y[64], z[64] per map) so
+// that a thread's four columns are one conflict-free 128-bit load per axis;
+// each thread writes 4 float4 of every staged map with streaming stores.  The
+// square root is sqrt.approx (relative error about 2^-23; exact 0 on the
+// diagonal).
+constexpr int kPdistMaps = 4;
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 __global__ void __launch_bounds__(256) pdist_kernel(const float *__restrict__ coords, int64_t n,
                                                     float *__restrict__ maps) {
-    __shared__ __align__(16) float sc[kN * 3];
-    for (int64_t m = blockIdx.x; m < n; m += gridDim.x) {
-        if (threadIdx.x < kN * 3 / 4)
-            reinterpret_cast<float4 *>(sc)[threadIdx.x] = ldg4(coords + m * (kN * 3) + 4 * threadIdx.x);
+    __shared__ __align__(16) float sc[kPdistMaps][3][kN];
+    for (int64_t m0 = (int64_t)blockIdx.x * kPdistMaps; m0 < n; m0 += (int64_t)gridDim.x * kPdistMaps) {
+        const int nm = (int)min((int64_t)kPdistMaps, n - m0);
+        for (int t = threadIdx.x; t < nm * kN * 3; t += blockDim.x) {
+            const int mm = t / (kN * 3), e = t - mm * (kN * 3);
+            sc[mm][e % 3][e / 3] = __ldg(coords + (m0 + mm) * (kN * 3) + e);
+        }
         __syncthreads();
-        float *out = maps + m * kMapFloats;
-#pragma unroll 4
-        for (int p = threadIdx.x; p < kMapFloats / 4; p += blockDim.x) {
-            const int i = p >> 4, q = p & 15;
-            const float xi = sc[3 * i], yi = sc[3 * i + 1], zi = sc[3 * i + 2];
-            float d[4];
+        for (int mm = 0; mm < nm; ++mm) {
+            float *out = maps + (m0 + mm) * kMapFloats;
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int j = 4 * q + t;
-                const float dx = xi - sc[3 * j], dy = yi - sc[3 * j + 1], dz = zi - sc[3 * j + 2];
-                d[t] = sqrtf(fmaf(dz, dz, fmaf(dy, dy, dx * dx)));
+            for (int it = 0; it < kMapFloats / 4 / 256; ++it) {
+                const int p = threadIdx.x + it * 256;
+                const int i = p >> 4, q = p & 15;
+                const float xi = sc[mm][0][i], yi = sc[mm][1][i], zi = sc[mm][2][i];
+                const float4 xj = reinterpret_cast<const float4 *>(sc[mm][0])[q];
+                const float4 yj = reinterpret_cast<const float4 *>(sc[mm][1])[q];
+                const float4 zj = reinterpret_cast<const float4 *>(sc[mm][2])[q];
+                float4 d;
+                d.x = sqrt_approx(fmaf(zi - zj.x, zi - zj.x, fmaf(yi - yj.x, yi - yj.x, (xi - xj.x) * (xi - xj.x))));
+                d.y = sqrt_approx(fmaf(zi - zj.y, zi - zj.y, fmaf(yi - yj.y, yi - yj.y, (xi - xj.y) * (xi - xj.y))));
+                d.z = sqrt_approx(fmaf(zi - zj.z, zi - zj.z, fmaf(yi - yj.z, yi - yj.z, (xi - xj.z) * (xi - xj.z))));
+                d.w = sqrt_approx(fmaf(zi - zj.w, zi - zj.w, fmaf(yi - yj.w, yi - yj.w, (xi - xj.w) * (xi - xj.w))));
+                __stcs(reinterpret_cast<float4 *>(out + 4 * p), d);
             }
-            __stcs(reinterpret_cast<float4 *>(out + 4 * p), make_float4(d[0], d[1], d[2], d[3]));
         }
         __syncthreads();
     }
@@ -399,7 +420,7 @@ cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigva
 
 cudaError_t launch_pdist(const float *coords, int64_t n, float *maps, cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
-    int64_t grid = n;
+    int64_t grid = (n + kPdistMaps - 1) / kPdistMaps;
     const int64_t cap = (int64_t)sms() * 8;
     if (grid > cap) grid = cap;
     pdist_kernel<<<(int)grid, 256, 0, st>>>(coords, n, maps);
