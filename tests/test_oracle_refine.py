@@ -1,5 +1,6 @@
 """Pins of the oracle's SMACOF refinement."""
 import numpy as np
+import pytest
 
 import synth
 from oracle import mds, refine
@@ -54,3 +55,56 @@ def test_refinement_reduces_stress_of_the_initialisation():
     s0 = refine.stress(X0, maps)
     _, s = refine.smacof(X0, maps, 30)
     assert np.all(s < s0)
+
+
+def test_transposed_maps_give_the_same_refinement():
+    # the map is symmetrised first, so D and D^T refine alike
+    g = np.random.default_rng(4)
+    pts = synth.random_points(7, 2, n=20)
+    D = synth.exact_distance_maps(pts) * (1 + 0.05 * g.standard_normal((2, 20, 20)))
+    X0 = pts + 0.2 * g.standard_normal(pts.shape)
+    Xa, sa = refine.smacof(X0, D, 8)
+    Xb, sb = refine.smacof(X0, np.swapaxes(D, 1, 2), 8)
+    np.testing.assert_allclose(Xa, Xb, atol=1e-12)
+    np.testing.assert_allclose(sa, sb, rtol=1e-12)
+
+
+_PINS = [test_guttman_step_is_a_gradient_step, test_stress_never_increases, test_exact_distances_are_a_fixed_point,
+         test_transposed_maps_give_the_same_refinement]
+
+
+@pytest.mark.parametrize("mistake", ["n_minus_1", "sign", "no_diagonal", "squared_weights", "no_symmetrise"])
+def test_pins_catch_planted_mistakes(mistake, monkeypatch):
+    # plant a plausible mistake in the oracle; at least one pin must fail
+    orig_gt = refine.guttman_transform
+
+    def bad_gt(X, D):
+        X = np.asarray(X, dtype=np.float64)
+        n = X.shape[-2]
+        d = refine.pairwise(X)
+        safe = np.where(d > 0.0, d, 1.0)
+        w = D / safe if mistake != "squared_weights" else (D / safe) ** 2
+        Bm = np.where(d > 0.0, -w if mistake != "sign" else w, 0.0)
+        idx = np.arange(n)
+        Bm[..., idx, idx] = 0.0
+        if mistake != "no_diagonal":
+            Bm[..., idx, idx] = -Bm.sum(axis=-1)
+        return Bm @ X / (n - 1 if mistake == "n_minus_1" else n)
+
+    def bad_smacof(X0, D, iterations):
+        X = np.asarray(X0, dtype=np.float64)
+        for _ in range(iterations):
+            X = orig_gt(X, np.asarray(D, dtype=np.float64))
+        return X, refine.stress(X, D)
+
+    if mistake == "no_symmetrise":
+        monkeypatch.setattr(refine, "smacof", bad_smacof)
+    else:
+        monkeypatch.setattr(refine, "guttman_transform", bad_gt)
+    failed = 0
+    for pin in _PINS:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, f"no pin caught {mistake}"
