@@ -110,6 +110,16 @@ const char *tdm_ctx_last_error(const tdm_ctx *ctx);
  * last call.  Returns TDM_ENOTCONVERGED when TDM_FLAG_MDS_NOT_CONVERGED was set. */
 tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out);
 
+/* The cosine alphas-bar table of Nichol & Dhariwal, "Improved Denoising
+ * Diffusion Probabilistic Models" (2021, section 3.2), for passing to
+ * tdm_init_schedule as alphas_bar_opt: alphas_bar(t) = f(t) / f(0),
+ * f(t) = cos^2(((t / T_train) + s) / (1 + s) * pi / 2), each beta clipped at
+ * 0.999; entry k is timestep k + 1.  ParaChromo §4.3.2 names a cosine schedule
+ * without its constants; s = 0.008 is the published offset.  Host function:
+ * alphas_bar_out is a host array [T_train].  Errors: TDM_EINVAL (T_train < 1,
+ * s < 0 or not finite, NULL output). */
+tdm_status tdm_cosine_alphas_bar(int32_t T_train, double s, double *alphas_bar_out);
+
 /* ---- schedule (ParaChromo §4.1, §5.1.1: reduced-step DDIM) --------------
  * Builds, in float64 on the host, beta_t linear from beta_start to beta_end
  * over T_train steps (or takes alphas_bar_opt[T_train] as given), the DDIM

@@ -35,6 +35,25 @@ def alphas_bar(betas: np.ndarray) -> np.ndarray:
     return out
 
 
+def cosine_alphas_bar(T_train: int = 1000, s: float = 0.008, max_beta: float = 0.999) -> np.ndarray:
+    """The cosine schedule of Nichol & Dhariwal, "Improved Denoising Diffusion
+    Probabilistic Models" (ICML 2021, section 3.2): alphas_bar(t) = f(t) / f(0)
+    with f(t) = cos^2(((t / T) + s) / (1 + s) * pi / 2), beta clipped at
+    max_beta.  Entry k of the table is timestep t = k + 1 (entry 0 is the first
+    noising step).  ParaChromo §4.3.2 names a cosine schedule; its constants
+    are not on the pages, so the published ones are used."""
+    def f(t):
+        return np.cos(((t / T_train) + s) / (1.0 + s) * np.pi / 2.0) ** 2
+
+    out = np.empty(T_train)
+    acc = 1.0
+    for k in range(T_train):
+        beta = min(1.0 - f(k + 1.0) / f(float(k)), max_beta)
+        acc *= 1.0 - beta
+        out[k] = acc
+    return out
+
+
 def ddim_timesteps(T_train: int, S: int) -> np.ndarray:
     if S < 1 or T_train % S != 0:
         raise ValueError("S must divide T_train")

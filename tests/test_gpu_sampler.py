@@ -38,6 +38,31 @@ def test_schedule_table_matches_oracle(tdm):
         np.testing.assert_allclose(tab[:, 3], o.sigma, rtol=1e-12, atol=1e-15)
 
 
+def test_cosine_schedule(tdm):
+    # the library's cosine table (Nichol & Dhariwal) against the oracle's, the
+    # DDIM table built from it, and a fused run on it
+    for T_train, s in ((1000, 0.008), (1200, 0.0), (7, 0.1)):
+        np.testing.assert_allclose(tdm.cosine_alphas_bar(T_train, s), osched.cosine_alphas_bar(T_train, s),
+                                   rtol=1e-13)
+    ab = tdm.cosine_alphas_bar(1000)
+    oab = osched.cosine_alphas_bar(1000)
+    for S, eta in ((50, 0.0), (250, 1.0)):
+        tab = np.array(tdm.Schedule(S, eta, alphas_bar=ab).table())
+        o = osched.Schedule(S=S, eta=eta, alphas_bar_table=oab)
+        np.testing.assert_array_equal(tab[:, 0], o.tau)
+        np.testing.assert_allclose(tab[:, 1], o.ab_t, rtol=1e-13)
+        np.testing.assert_allclose(tab[:, 2], o.ab_p, rtol=1e-13)
+        np.testing.assert_allclose(tab[:, 3], o.sigma, rtol=1e-11, atol=1e-15)
+    t = tdm.Tiling(C=1, T=4, B=8, overlap=12, sync_every=1)
+    x0 = synth.chain_x0(0, 1, 4)
+    maps = _maps(t)
+    tdm.ddim_run(tdm.Schedule(50, eta=1.0, alphas_bar=ab), maps, dev(x0), 1.0, 0.1, 0.3, 0, t)
+    ref = o_run(x0, osched.Schedule(S=50, eta=1.0, alphas_bar_table=oab), 1.0, 0.1, 0.3, 0, np.arange(8), 8)
+    assert_maps_close(_as5(maps, t), ref, TOL_MAP, "fused run on the cosine schedule")
+    with pytest.raises(tdm.TdmError):
+        tdm.cosine_alphas_bar(0)
+
+
 @pytest.mark.parametrize("base,boff", [(0, 0), (12345, 3)])
 def test_init_noise(tdm, base, boff):
     t = tdm.Tiling(C=2, T=3, B=4, B_total=9, b_offset=boff, sample_id_base=base)

@@ -69,3 +69,26 @@ def test_ddim_preserves_forward_marginal_form(eta):
         out = ddim_update(xt, e, s.ab_t[i], s.ab_p[i], s.sigma[i], np.zeros_like(e))
         ref = np.sqrt(s.ab_p[i]) * x0 + np.sqrt(1 - s.ab_p[i] - s.sigma[i] ** 2) * e
         np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_cosine_schedule_closed_forms():
+    # with s = 0 and no beta reaching the clip, alphas_bar(t) telescopes to
+    # cos^2(pi t / 2T): 1/2 at t = T/2 and 3/4 at t = T/3 (entry t - 1)
+    ab = schedule.cosine_alphas_bar(1200, s=0.0)
+    assert ab[600 - 1] == pytest.approx(0.5, rel=1e-12)
+    assert ab[400 - 1] == pytest.approx(0.75, rel=1e-12)
+    assert ab[0] == pytest.approx(np.cos(np.pi / 2400) ** 2, rel=1e-14)
+
+
+def test_cosine_schedule_clip_and_order():
+    ab = schedule.cosine_alphas_bar(1000)
+    assert np.all(np.diff(ab) < 0) and ab[0] < 1.0 and ab[-1] > 0.0
+    betas = 1.0 - ab / np.concatenate([[1.0], ab[:-1]])
+    assert betas[-1] == pytest.approx(0.999, rel=1e-12)     # f(T) = 0 is clipped
+    assert betas.max() <= 0.999 + 1e-12
+    # the offset s keeps the first beta small: 1 - f(1)/f(0) for s = 0.008
+    f = lambda t: np.cos((t / 1000 + 0.008) / 1.008 * np.pi / 2) ** 2
+    assert betas[0] == pytest.approx(1 - f(1) / f(0), rel=1e-12)
+    # a schedule built from the table accepts it as given
+    sch = schedule.Schedule(S=50, alphas_bar_table=ab)
+    np.testing.assert_allclose(sch.ab_t, ab[::20])

@@ -65,6 +65,7 @@ _SIGS = {
     "tdm_kabsch_stitch": (_i32, [_vp, _vp, _P(CTiling), _vp, _vp, _vp]),
     "tdm_refine_smacof": (_i32, [_vp, _vp, _i64, _vp, _i32, _vp, _vp]),
     "tdm_nonoverlap_drift": (_i32, [_vp, _vp, _vp, _P(CTiling), _vp, _vp, _vp]),
+    "tdm_cosine_alphas_bar": (_i32, [_i32, _f64, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -355,6 +356,16 @@ def nonoverlap_drift(maps, ref, tiling: Tiling, tile_sums_out, drift_out=None, c
                                         _ptr(tile_sums_out, "tile_sums_out", ctx), _ptr(drift_out, "drift_out", ctx),
                                         _stream(ctx)))
     return tile_sums_out
+
+
+def cosine_alphas_bar(T_train: int = 1000, s: float = 0.008) -> list[float]:
+    """The cosine alphas-bar table (Nichol & Dhariwal 2021) for
+    ``Schedule(..., alphas_bar=...)`` (see tdm_cosine_alphas_bar)."""
+    out = (_f64 * int(T_train))()
+    st = _lib.tdm_cosine_alphas_bar(int(T_train), float(s), ctypes.cast(out, ctypes.c_void_p))
+    if st != OK:
+        raise TdmError(st, "cosine_alphas_bar: T_train >= 1 and s >= 0 required")
+    return list(out)
 
 
 def kabsch_stitch(coords, tiling: Tiling, chain_out, residual_out=None, ctx: Context | None = None):

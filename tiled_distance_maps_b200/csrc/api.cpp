@@ -1,5 +1,6 @@
 // extern "C" entry points of libtdm: argument validation, context, schedule,
 // and dispatch to the kernel launchers.  See include/tdm.h for the contract.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -164,6 +165,25 @@ tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out) {
 }
 
 // ---- schedule -----------------------------------------------------------------------
+
+tdm_status tdm_cosine_alphas_bar(int32_t T_train, double s, double *alphas_bar_out) {
+    if (T_train < 1 || !(s >= 0.0) || !std::isfinite(s) || alphas_bar_out == nullptr) return TDM_EINVAL;
+    constexpr double kHalfPi = 1.5707963267948966;
+    constexpr double kMaxBeta = 0.999;
+    auto f = [&](double t) {
+        const double c = std::cos((t / (double)T_train + s) / (1.0 + s) * kHalfPi);
+        return c * c;
+    };
+    double acc = 1.0, f_prev = f(0.0);
+    for (int k = 0; k < T_train; ++k) {
+        const double f_next = f((double)k + 1.0);
+        const double beta = std::min(1.0 - f_next / f_prev, kMaxBeta);
+        acc *= 1.0 - beta;
+        alphas_bar_out[k] = acc;
+        f_prev = f_next;
+    }
+    return TDM_OK;
+}
 
 tdm_status tdm_init_schedule(tdm_ctx *ctx, tdm_schedule **out, int32_t T_train, double beta_start,
                              double beta_end, const double *alphas_bar_opt, int32_t S, double eta) {
