@@ -187,6 +187,18 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
                         float s_c, float s_u, uint64_t seed, int32_t init_noise,
                         const tdm_tiling *tiling, tdm_stream stream);
 
+/* Part of the same run: steps first_step, first_step - 1, .., first_step -
+ * n_steps + 1 (0 <= first_step < S, 1 <= n_steps <= first_step + 1), with the
+ * state read from maps (or x_T drawn when init_noise != 0, allowed only for
+ * first_step = S-1) and written back.  The noise is keyed by the step index
+ * and the projection follows the steps counted from step S-1, so a run split
+ * into parts (the state kept in maps in between, e.g. saved and restored as a
+ * checkpoint) gives the same maps, bit for bit, as the whole run.  Errors as
+ * tdm_ddim_run, plus TDM_EINVAL for a step range outside the schedule. */
+tdm_status tdm_ddim_run_steps(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w,
+                              float s_c, float s_u, uint64_t seed, int32_t init_noise, int32_t first_step,
+                              int32_t n_steps, const tdm_tiling *tiling, tdm_stream stream);
+
 /* Overlap-consistency projection, in place (ParaChromo §4.3.2, Algorithm 1):
  * for every chain c, seam k < T-1 and sample b, M = 0.5 * (right block of tile
  * k + left block of tile k+1), the blocks being rows/cols [64-o, 64) and

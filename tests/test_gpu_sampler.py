@@ -282,3 +282,32 @@ def test_ddpm_ancestral_sampler_1000_steps(tdm):
         x = ddpm_ancestral_step(x, 2.0 * ec - eu, tt, o.betas, o.ab, stream_noise(23, philox.TAG_ETA, tt, g))
         x = seam_project(x)
     assert_maps_close(_as5(maps, t), x, TOL_MAP, "DDPM run")
+
+
+@pytest.mark.parametrize("S,K,eta,w,cuts", [(10, 1, 0.0, 1.0, (4,)), (10, 3, 1.0, 0.0, (2, 7)),
+                                            (8, 0, 0.0, 1.0, (5,)), (20, 3, 1.0, 1.0, (1, 10, 19))])
+def test_fused_run_resumes_bit_exactly(tdm, S, K, eta, w, cuts):
+    # the run split after the given numbers of steps, the state kept in the
+    # maps between the parts, equals the whole run bit for bit
+    t = tdm.Tiling(C=2, T=3, B=4, overlap=12, sync_every=K)
+    sch = tdm.Schedule(S, eta=eta)
+    x0 = dev(synth.chain_x0(2, 2, 3)).reshape(-1)
+    whole = _maps(t)
+    tdm.ddim_run(sch, whole, x0, w, 0.1, 0.3, 9, t)
+    parts = _maps(t)
+    done = 0
+    for n in list(cuts) + [S]:
+        tdm.ddim_run(sch, parts, x0, w, 0.1, 0.3, 9, t, init_noise=done == 0, first_step=S - 1 - done,
+                     n_steps=n - done)
+        done = n
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(parts), host(whole))
+
+
+def test_fused_run_step_range_is_checked(tdm):
+    t = tdm.Tiling(C=1, T=2, B=1)
+    sch = tdm.Schedule(10)
+    x0, m = dev(synth.chain_x0(0, 1, 2)).reshape(-1), _maps(t)
+    for first, n, init in ((10, 1, False), (-1, 1, False), (5, 7, False), (5, 0, False), (5, 2, True)):
+        with pytest.raises(tdm.TdmError):
+            tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.0, 0, t, init_noise=init, first_step=first, n_steps=n)

@@ -53,6 +53,7 @@ _SIGS = {
     "tdm_eps_standin": (_i32, [_vp, _vp, _i32, _vp, _vp, _f32, _i32, _u64, _P(CTiling), _vp, _vp]),
     "tdm_ddim_step": (_i32, [_vp, _vp, _i32, _vp, _vp, _vp, _f32, _u64, _P(CTiling), _vp]),
     "tdm_ddim_run": (_i32, [_vp, _vp, _vp, _vp, _f32, _f32, _f32, _u64, _i32, _P(CTiling), _vp]),
+    "tdm_ddim_run_steps": (_i32, [_vp, _vp, _vp, _vp, _f32, _f32, _f32, _u64, _i32, _i32, _i32, _P(CTiling), _vp]),
     "tdm_seam_project": (_i32, [_vp, _vp, _P(CTiling), _vp]),
     "tdm_mds_recover": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp]),
     "tdm_pairwise_dist": (_i32, [_vp, _vp, _i64, _vp, _vp]),
@@ -263,14 +264,22 @@ def ddim_step(sched: Schedule, step: int, maps, eps_c, eps_u, w: float, seed: in
 
 
 def ddim_run(sched: Schedule, maps, x0, w: float, s_c: float, s_u: float, seed: int, tiling: Tiling,
-             init_noise: bool = True, ctx: Context | None = None):
+             init_noise: bool = True, ctx: Context | None = None, first_step: int | None = None,
+             n_steps: int | None = None):
+    """The fused reverse run (tdm_ddim_run); with ``first_step`` / ``n_steps``
+    only that part of it (tdm_ddim_run_steps), e.g. to resume from saved maps."""
     ctx = ctx or sched.ctx
     _need(maps, tiling.n_maps * 4096, "maps")
     _need(x0, tiling.C * tiling.T * 4096, "x0")
     ct = tiling.c()
-    ctx.check(_lib.tdm_ddim_run(ctx.handle, sched.handle, _ptr(maps, "maps", ctx), _ptr(x0, "x0", ctx), float(w),
-                                float(s_c), float(s_u), int(seed), 1 if init_noise else 0, ctypes.byref(ct),
-                                _stream(ctx)))
+    args = (ctx.handle, sched.handle, _ptr(maps, "maps", ctx), _ptr(x0, "x0", ctx), float(w), float(s_c),
+            float(s_u), int(seed), 1 if init_noise else 0)
+    if first_step is None and n_steps is None:
+        ctx.check(_lib.tdm_ddim_run(*args, ctypes.byref(ct), _stream(ctx)))
+    else:
+        first = sched.S - 1 if first_step is None else int(first_step)
+        count = first + 1 if n_steps is None else int(n_steps)
+        ctx.check(_lib.tdm_ddim_run_steps(*args, first, count, ctypes.byref(ct), _stream(ctx)))
     return maps
 
 

@@ -357,6 +357,21 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
     if (ctx == nullptr) return TDM_EINVAL;
     tdm_status s = check_sched(ctx, sched);
     if (s != TDM_OK) return s;
+    return tdm_ddim_run_steps(ctx, sched, maps, x0, w, s_c, s_u, seed, init_noise, sched->S - 1, sched->S, tiling,
+                              stream);
+}
+
+tdm_status tdm_ddim_run_steps(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w,
+                              float s_c, float s_u, uint64_t seed, int32_t init_noise, int32_t first_step,
+                              int32_t n_steps, const tdm_tiling *tiling, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    tdm_status s = check_sched(ctx, sched);
+    if (s != TDM_OK) return s;
+    if (first_step < 0 || first_step >= sched->S || n_steps < 1 || n_steps > first_step + 1)
+        return fail(ctx, TDM_EINVAL, "ddim_run: need 0 <= first_step < S and 1 <= n_steps <= first_step + 1 "
+                                     "(got %d, %d, S = %d)", first_step, n_steps, sched->S);
+    if (init_noise != 0 && first_step != sched->S - 1)
+        return fail(ctx, TDM_EINVAL, "ddim_run: init_noise draws x_T, the state before step S-1 only");
     Tiling t;
     if ((s = check_tiling(ctx, tiling, &t)) != TDM_OK) return s;
     if (!std::isfinite(w) || !std::isfinite(s_c) || !std::isfinite(s_u))
@@ -386,8 +401,9 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
             ctx->plans[{t.T, ov}] = plan;
         }
     }
-    cudaError_t e = tdm::launch_ddim_run(sched->d_coef, sched->S, maps, x0, w, s_c, s_u, sched->eta > 0.0, seed,
-                                         init_noise != 0, t, plan, static_cast<cudaStream_t>(stream));
+    cudaError_t e = tdm::launch_ddim_run(sched->d_coef, sched->S, first_step, n_steps, maps, x0, w, s_c, s_u,
+                                         sched->eta > 0.0, seed, init_noise != 0, t, plan,
+                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "ddim_run launch");
 }
 

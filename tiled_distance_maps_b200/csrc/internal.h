@@ -64,9 +64,9 @@ cudaError_t launch_eps_standin(const StepCoef *coef, int step, const float *maps
 cudaError_t launch_ddim_step(const StepCoef *coef, int step, float *maps, const float *eps_c,
                              const float *eps_u, float w, bool has_eta, uint64_t seed, const Tiling &t,
                              cudaStream_t st);
-cudaError_t launch_ddim_run(const StepCoef *coef, int S, float *maps, const float *x0, float w, float s_c,
-                            float s_u, bool has_eta, uint64_t seed, bool init_noise, const Tiling &t,
-                            const uint32_t *plan, cudaStream_t st);
+cudaError_t launch_ddim_run(const StepCoef *coef, int S, int first, int n_steps, float *maps, const float *x0,
+                            float w, float s_c, float s_u, bool has_eta, uint64_t seed, bool init_noise,
+                            const Tiling &t, const uint32_t *plan, cudaStream_t st);
 cudaError_t launch_seam_project(float *maps, const Tiling &t, cudaStream_t st);
 cudaError_t launch_seam_sums(const float *maps, const Tiling &t, float *partial, int chunks,
                              cudaStream_t st);

@@ -170,6 +170,7 @@ struct RunArgs {
     int64_t total_warps;       // C * B * 17 T
     int64_t B_total, b_off, base;
     int S, T, B, sync_every, warps_per_chain;
+    int first, last;           // steps first, first-1, .., last (first = S-1, last = 0 for a whole run)
     float cc, cu;              // (1 + w) s_c and w s_u
     PhiloxKeys K;
 };
@@ -248,7 +249,9 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     // the plan) take part in the projection
     const bool warp_pairs = __shfl_sync(0xffffffffu, paired ? 1 : 0, 0) != 0;
     const bool sync_warp = a.T > 1 && a.sync_every > 0 && warp_pairs;
-    int until_sync = a.sync_every;
+    // the projection follows the steps counted from the start of the whole
+    // run, so a run resumed at step `first` projects where the whole run would
+    int until_sync = a.sync_every > 0 ? a.sync_every - (a.S - 1 - a.first) % a.sync_every : 0;
 
     constexpr int NS = 1 + (HAS_U ? 1 : 0) + (HAS_ETA ? 1 : 0);
     constexpr int kTags[3] = {TDM_STREAM_EPS_C, HAS_U ? TDM_STREAM_EPS_U : TDM_STREAM_ETA, TDM_STREAM_ETA};
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
 #pragma unroll
     for (int s = 0; s < NS; ++s) tags[s] = kTags[s];
 
-    for (int i = a.S - 1; i >= 0; --i) {
+    for (int i = a.first; i >= a.last; --i) {
         const float4 cf = sco[i];
         float4 z[NS];
         lane_normals<NS>(L, (uint32_t)i, tags, a.K, z);
@@ -423,10 +426,12 @@ static cudaError_t run_variant(const RunArgs &a, int grid, size_t smem, cudaStre
     return cudaGetLastError();
 }
 
-cudaError_t launch_ddim_run(const StepCoef *coef, int S, float *maps, const float *x0, float w, float s_c,
-                            float s_u, bool has_eta, uint64_t seed, bool init_noise, const Tiling &t,
-                            const uint32_t *plan, cudaStream_t st) {
+cudaError_t launch_ddim_run(const StepCoef *coef, int S, int first, int n_steps, float *maps, const float *x0,
+                            float w, float s_c, float s_u, bool has_eta, uint64_t seed, bool init_noise,
+                            const Tiling &t, const uint32_t *plan, cudaStream_t st) {
     RunArgs a;
+    a.first = first;
+    a.last = first - n_steps + 1;
     a.coef = coef;
     a.maps = maps;
     a.x0 = x0;
