@@ -47,7 +47,7 @@ typedef int32_t tdm_status;
 #define TDM_EINVAL         1  /* bad argument (null, misaligned, out of range) */
 #define TDM_ECUDA          2  /* a CUDA runtime call or launch failed */
 #define TDM_ETIMEOUT       3  /* reserved: no kernel of this library waits on another */
-#define TDM_ENONFINITE     4  /* reserved for a non-finite scan of outputs */
+#define TDM_ENONFINITE     4  /* tdm_scan_nonfinite found NaN or inf (see tdm_ctx_sync) */
 #define TDM_EUNSUPPORTED   5  /* valid request this build does not implement */
 #define TDM_ENOMEM         6  /* device allocation failed */
 #define TDM_ENOTCONVERGED  7  /* an MDS eigen-solve hit its iteration cap (see tdm_ctx_sync) */
@@ -60,6 +60,7 @@ typedef int32_t tdm_status;
 
 /* device status flags returned by tdm_ctx_sync */
 #define TDM_FLAG_MDS_NOT_CONVERGED 0x1u
+#define TDM_FLAG_NONFINITE         0x2u   /* raised by tdm_scan_nonfinite */
 
 /* columns of the host schedule table (tdm_schedule_table), one row per DDIM step i */
 #define TDM_SCHED_COLS 8   /* tau_i, ab_t, ab_p, sigma_i, a_i, b_i, sqrt(ab_t), 1/sqrt(1-ab_t) */
@@ -107,8 +108,17 @@ const char *tdm_ctx_last_error(const tdm_ctx *ctx);
 
 /* Synchronises `stream`, then reads and clears the context's device status
  * word.  *flags_out (may be NULL) receives the TDM_FLAG_* bits raised since the
- * last call.  Returns TDM_ENOTCONVERGED when TDM_FLAG_MDS_NOT_CONVERGED was set. */
+ * last call.  Returns TDM_ENONFINITE when TDM_FLAG_NONFINITE was set, else
+ * TDM_ENOTCONVERGED when TDM_FLAG_MDS_NOT_CONVERGED was set. */
 tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out);
+
+/* Scans buf[0 .. n) (device floats, 4-byte aligned, read only) on `stream`
+ * and raises TDM_FLAG_NONFINITE in the context's status word when any value
+ * is NaN or +-inf; the result is read by tdm_ctx_sync.  Meant for a caller's
+ * check of any output (the library's kernels never produce non-finite values
+ * from finite inputs).  Errors: TDM_EINVAL (NULL ctx, n < 0, NULL or
+ * misaligned buf with n > 0). */
+tdm_status tdm_scan_nonfinite(tdm_ctx *ctx, const float *buf, int64_t n, tdm_stream stream);
 
 /* The cosine alphas-bar table of Nichol & Dhariwal, "Improved Denoising
  * Diffusion Probabilistic Models" (2021, section 3.2), for passing to

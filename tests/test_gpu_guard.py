@@ -112,3 +112,22 @@ def test_noise_primitives_stay_in_bounds(tdm):
     z = Guarded(4 * n)             # 4n words = 2n pairs = 4n normals
     tdm.box_muller(out.t, z.t)
     assert z.intact(), "box_muller"
+
+
+@pytest.mark.parametrize("n,off", [(1, 0), (4099, 1), (1 << 20, 3), (7, 2)])
+def test_nonfinite_scan(tdm, n, off):
+    # a clean buffer raises nothing; one NaN or inf anywhere (head, body or
+    # tail of the vectorised range, at any offset from 16-byte alignment) does
+    base = torch.randn(n + 8, device="cuda")
+    buf = base[off:off + n]
+    tdm.scan_nonfinite(buf)
+    assert tdm.ctx_sync() == 0
+    for pos in sorted({0, n // 2, n - 1}):
+        for bad in (float("nan"), float("inf"), float("-inf")):
+            buf[pos] = bad
+            tdm.scan_nonfinite(buf)
+            assert tdm.ctx_sync() & tdm.FLAG_NONFINITE, (pos, bad)
+            buf[pos] = 1.0
+    base[off + n] = float("nan")            # just past the end: not scanned
+    tdm.scan_nonfinite(buf)
+    assert tdm.ctx_sync() == 0

@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, EINVAL, ECUDA, ETIMEOUT, ENONFINITE, EUNSUPPORTED, ENOMEM, ENOTCONVERGED = range(8)
 STREAM_INIT, STREAM_EPS_C, STREAM_EPS_U, STREAM_ETA = range(4)
 FLAG_MDS_NOT_CONVERGED = 0x1
+FLAG_NONFINITE = 0x2
 SCHED_COLS = 8
 
 _c = ctypes
@@ -67,6 +68,7 @@ _SIGS = {
     "tdm_refine_smacof": (_i32, [_vp, _vp, _i64, _vp, _i32, _vp, _vp]),
     "tdm_nonoverlap_drift": (_i32, [_vp, _vp, _vp, _P(CTiling), _vp, _vp, _vp]),
     "tdm_cosine_alphas_bar": (_i32, [_i32, _f64, _vp]),
+    "tdm_scan_nonfinite": (_i32, [_vp, _vp, _i64, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -446,6 +448,15 @@ def ctx_sync(ctx: Context | None = None) -> int:
     ctx = ctx or context()
     flags = ctypes.c_uint32(0)
     st = _lib.tdm_ctx_sync(ctx.handle, _stream(ctx), ctypes.byref(flags))
-    if st not in (OK, ENOTCONVERGED):
+    if st not in (OK, ENOTCONVERGED, ENONFINITE):
         ctx.check(st)
     return flags.value
+
+
+def scan_nonfinite(buf, ctx: Context | None = None):
+    """Raise FLAG_NONFINITE (read by ctx_sync) when the float32 CUDA tensor
+    ``buf`` holds NaN or inf (see tdm_scan_nonfinite)."""
+    import torch
+    ctx = ctx or context(buf.device.index)
+    ctx.check(_lib.tdm_scan_nonfinite(ctx.handle, _uptr(buf, "buf", ctx, torch.float32), int(buf.numel()),
+                                      _stream(ctx)))

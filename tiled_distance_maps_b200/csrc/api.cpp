@@ -159,9 +159,21 @@ tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out) {
     if (e == cudaSuccess) e = cudaMemset(ctx->d_flags, 0, sizeof(uint32_t));
     if (e != cudaSuccess) return cuda_fail(ctx, e, "status word");
     if (flags_out != nullptr) *flags_out = flags;
+    if (flags & TDM_FLAG_NONFINITE) return fail(ctx, TDM_ENONFINITE, "a scanned buffer held NaN or inf");
     if (flags & TDM_FLAG_MDS_NOT_CONVERGED)
         return fail(ctx, TDM_ENOTCONVERGED, "an MDS eigen-solve reached its iteration cap");
     return TDM_OK;
+}
+
+tdm_status tdm_scan_nonfinite(tdm_ctx *ctx, const float *buf, int64_t n, tdm_stream stream) {
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (n < 0) return fail(ctx, TDM_EINVAL, "scan: n < 0");
+    if (n == 0) return TDM_OK;
+    if (buf == nullptr || (reinterpret_cast<uintptr_t>(buf) & 3u))
+        return fail(ctx, TDM_EINVAL, "scan: buf is NULL or not 4-byte aligned");
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_scan_nonfinite(buf, n, ctx->d_flags, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "scan launch");
 }
 
 // ---- schedule -----------------------------------------------------------------------

@@ -88,6 +88,7 @@ cudaError_t launch_box_muller(const uint32_t *words, int64_t n_pairs, float *z, 
 std::vector<uint32_t> build_run_plan(int T, int overlap);
 int seam_chunks(int64_t n_seams, int B);
 int drift_chunks(int64_t tiles, int B);
+cudaError_t launch_scan_nonfinite(const float *buf, int64_t n, uint32_t *flags, cudaStream_t st);
 cudaError_t launch_drift(const float *S, const float *V, const Tiling &t, float *scratch, int chunks,
                          float *tile_sums, float *drift, cudaStream_t st);
 
