@@ -7,6 +7,8 @@
 #include <cstring>
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 
 using tdm::StepCoef;
@@ -90,6 +92,15 @@ tdm_status check_sched(tdm_ctx *ctx, const tdm_schedule *s) {
 
 }  // namespace
 
+
+// An NVTX range around each entry point (a no-op unless a profiler is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
 extern "C" {
 
 const char *tdm_status_str(tdm_status s) {
@@ -109,6 +120,7 @@ const char *tdm_status_str(tdm_status s) {
 const char *tdm_ctx_last_error(const tdm_ctx *ctx) { return ctx == nullptr ? "" : ctx->last_error.c_str(); }
 
 tdm_status tdm_ctx_create(tdm_ctx **out, int32_t device) {
+    NvtxRange nvtx_range_("tdm_ctx_create");
     if (out == nullptr) return TDM_EINVAL;
     *out = nullptr;
     int count = 0;
@@ -149,6 +161,7 @@ void tdm_ctx_destroy(tdm_ctx *ctx) {
 }
 
 tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out) {
+    NvtxRange nvtx_range_("tdm_ctx_sync");
     if (ctx == nullptr) return TDM_EINVAL;
     DeviceScope ds(ctx->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -166,6 +179,7 @@ tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out) {
 }
 
 tdm_status tdm_scan_nonfinite(tdm_ctx *ctx, const float *buf, int64_t n, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_scan_nonfinite");
     if (ctx == nullptr) return TDM_EINVAL;
     if (n < 0) return fail(ctx, TDM_EINVAL, "scan: n < 0");
     if (n == 0) return TDM_OK;
@@ -199,6 +213,7 @@ tdm_status tdm_cosine_alphas_bar(int32_t T_train, double s, double *alphas_bar_o
 
 tdm_status tdm_init_schedule(tdm_ctx *ctx, tdm_schedule **out, int32_t T_train, double beta_start,
                              double beta_end, const double *alphas_bar_opt, int32_t S, double eta) {
+    NvtxRange nvtx_range_("tdm_init_schedule");
     if (ctx == nullptr || out == nullptr) return fail(ctx, TDM_EINVAL, "ctx or out is NULL");
     *out = nullptr;
     if (T_train < 1 || S < 1 || S > T_train || T_train % S != 0)
@@ -282,6 +297,7 @@ void tdm_schedule_destroy(tdm_schedule *s) {
 }
 
 tdm_status tdm_schedule_table(const tdm_schedule *s, double *out, int64_t n) {
+    NvtxRange nvtx_range_("tdm_schedule_table");
     if (s == nullptr || out == nullptr || n < (int64_t)s->table.size()) return TDM_EINVAL;
     std::memcpy(out, s->table.data(), s->table.size() * sizeof(double));
     return TDM_OK;
@@ -292,6 +308,7 @@ int32_t tdm_schedule_steps(const tdm_schedule *s) { return s == nullptr ? 0 : s-
 // ---- sampler ------------------------------------------------------------------------
 
 tdm_status tdm_init_noise(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, uint64_t seed, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_init_noise");
     if (ctx == nullptr) return TDM_EINVAL;
     Tiling t;
     tdm_status s = check_tiling(ctx, tiling, &t);
@@ -306,6 +323,7 @@ tdm_status tdm_init_noise(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, u
 tdm_status tdm_eps_standin(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, const float *maps,
                            const float *x0, float s_noise, int32_t stream_tag, uint64_t seed,
                            const tdm_tiling *tiling, float *eps_out, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_eps_standin");
     if (ctx == nullptr) return TDM_EINVAL;
     tdm_status s = check_sched(ctx, sched);
     if (s != TDM_OK) return s;
@@ -327,6 +345,7 @@ tdm_status tdm_eps_standin(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step
 }
 
 tdm_status tdm_seam_project(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_seam_project");
     if (ctx == nullptr) return TDM_EINVAL;
     Tiling t;
     tdm_status s = check_tiling(ctx, tiling, &t);
@@ -340,6 +359,7 @@ tdm_status tdm_seam_project(tdm_ctx *ctx, float *maps, const tdm_tiling *tiling,
 
 tdm_status tdm_ddim_step(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, float *maps, const float *eps_c,
                          const float *eps_u, float w, uint64_t seed, const tdm_tiling *tiling, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_ddim_step");
     if (ctx == nullptr) return TDM_EINVAL;
     tdm_status s = check_sched(ctx, sched);
     if (s != TDM_OK) return s;
@@ -366,6 +386,7 @@ tdm_status tdm_ddim_step(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, 
 
 tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w, float s_c,
                         float s_u, uint64_t seed, int32_t init_noise, const tdm_tiling *tiling, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_ddim_run");
     if (ctx == nullptr) return TDM_EINVAL;
     tdm_status s = check_sched(ctx, sched);
     if (s != TDM_OK) return s;
@@ -376,6 +397,7 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
 tdm_status tdm_ddim_run_steps(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w,
                               float s_c, float s_u, uint64_t seed, int32_t init_noise, int32_t first_step,
                               int32_t n_steps, const tdm_tiling *tiling, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_ddim_run_steps");
     if (ctx == nullptr) return TDM_EINVAL;
     tdm_status s = check_sched(ctx, sched);
     if (s != TDM_OK) return s;
@@ -423,6 +445,7 @@ tdm_status tdm_ddim_run_steps(tdm_ctx *ctx, const tdm_schedule *sched, float *ma
 
 tdm_status tdm_refine_smacof(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, int32_t iterations,
                              float *stress_out, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_refine_smacof");
     if (ctx == nullptr) return TDM_EINVAL;
     if (n_maps < 0) return fail(ctx, TDM_EINVAL, "n_maps < 0");
     if (iterations < 0) return fail(ctx, TDM_EINVAL, "iterations < 0");
@@ -440,6 +463,7 @@ tdm_status tdm_refine_smacof(tdm_ctx *ctx, const float *maps, int64_t n_maps, fl
 
 tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling *tiling, float *chain_out,
                              float *residual_out, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_kabsch_stitch");
     if (ctx == nullptr) return TDM_EINVAL;
     Tiling t;
     tdm_status s = check_tiling(ctx, tiling, &t);
@@ -460,6 +484,7 @@ tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling
 
 tdm_status tdm_philox4x32(tdm_ctx *ctx, const uint32_t *ctr, int64_t n, uint64_t seed, uint32_t *out,
                           tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_philox4x32");
     if (ctx == nullptr) return TDM_EINVAL;
     if (n < 0) return fail(ctx, TDM_EINVAL, "n < 0");
     if (n == 0) return TDM_OK;
@@ -471,6 +496,7 @@ tdm_status tdm_philox4x32(tdm_ctx *ctx, const uint32_t *ctr, int64_t n, uint64_t
 }
 
 tdm_status tdm_box_muller(tdm_ctx *ctx, const uint32_t *words, int64_t n_pairs, float *z, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_box_muller");
     if (ctx == nullptr) return TDM_EINVAL;
     if (n_pairs < 0) return fail(ctx, TDM_EINVAL, "n_pairs < 0");
     if (n_pairs == 0) return TDM_OK;
@@ -486,6 +512,7 @@ tdm_status tdm_box_muller(tdm_ctx *ctx, const uint32_t *words, int64_t n_pairs, 
 
 tdm_status tdm_mds_recover(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, float *eigvals_opt,
                            tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_mds_recover");
     if (ctx == nullptr) return TDM_EINVAL;
     if (n_maps < 0) return fail(ctx, TDM_EINVAL, "n_maps < 0");
     if (n_maps == 0) return TDM_OK;
@@ -499,6 +526,7 @@ tdm_status tdm_mds_recover(tdm_ctx *ctx, const float *maps, int64_t n_maps, floa
 }
 
 tdm_status tdm_pairwise_dist(tdm_ctx *ctx, const float *coords, int64_t n_maps, float *maps_out, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_pairwise_dist");
     if (ctx == nullptr) return TDM_EINVAL;
     if (n_maps < 0) return fail(ctx, TDM_EINVAL, "n_maps < 0");
     if (n_maps == 0) return TDM_OK;
@@ -512,6 +540,7 @@ tdm_status tdm_pairwise_dist(tdm_ctx *ctx, const float *coords, int64_t n_maps, 
 
 tdm_status tdm_seam_overlap_sums(tdm_ctx *ctx, const float *maps, const tdm_tiling *tiling, float *sums,
                                  tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_seam_overlap_sums");
     if (ctx == nullptr) return TDM_EINVAL;
     Tiling t;
     tdm_status s = check_tiling(ctx, tiling, &t);
@@ -541,6 +570,7 @@ tdm_status tdm_seam_overlap_sums(tdm_ctx *ctx, const float *maps, const tdm_tili
 
 tdm_status tdm_seam_discrepancy_finalize(tdm_ctx *ctx, const float *sums, const tdm_tiling *tiling, float *out,
                                          tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_seam_discrepancy_finalize");
     if (ctx == nullptr) return TDM_EINVAL;
     Tiling t;
     tdm_status s = check_tiling(ctx, tiling, &t);
@@ -557,6 +587,7 @@ tdm_status tdm_seam_discrepancy_finalize(tdm_ctx *ctx, const float *sums, const 
 
 tdm_status tdm_seam_discrepancy(tdm_ctx *ctx, const float *maps, const tdm_tiling *tiling, float *out,
                                 tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_seam_discrepancy");
     if (ctx == nullptr) return TDM_EINVAL;
     Tiling t;
     tdm_status s = check_tiling(ctx, tiling, &t);
@@ -583,6 +614,7 @@ tdm_status tdm_seam_discrepancy(tdm_ctx *ctx, const float *maps, const tdm_tilin
 
 tdm_status tdm_nonoverlap_drift(tdm_ctx *ctx, const float *maps, const float *ref, const tdm_tiling *tiling,
                                 float *tile_sums_out, float *drift_out, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_nonoverlap_drift");
     if (ctx == nullptr) return TDM_EINVAL;
     Tiling t;
     tdm_status s = check_tiling(ctx, tiling, &t);
