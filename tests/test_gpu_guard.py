@@ -131,3 +131,31 @@ def test_nonfinite_scan(tdm, n, off):
     base[off + n] = float("nan")            # just past the end: not scanned
     tdm.scan_nonfinite(buf)
     assert tdm.ctx_sync() == 0
+
+
+@pytest.mark.parametrize("C,T,B", [(0, 3, 4), (2, 3, 0)])
+def test_empty_inputs_write_nothing(tdm, C, T, B):
+    # no maps: every entry point returns without touching its (guard-only) outputs
+    t = tdm.Tiling(C=C, T=T, B=B, overlap=12, sync_every=1)
+    sch = tdm.Schedule(10)
+    x0 = torch.zeros(max(C, 1) * T * 4096, device="cuda")
+    band = Guarded(0)
+    tdm.init_noise(band.t, t, 1)
+    tdm.eps_standin(sch, 3, band.t, x0, 0.1, tdm.STREAM_EPS_C, 1, t, band.t)
+    tdm.ddim_step(sch, 3, band.t, band.t, band.t, 1.0, 1, t)
+    tdm.ddim_run(sch, band.t, x0, 1.0, 0.1, 0.3, 1, t)
+    tdm.seam_project(band.t, t)
+    seams, tiles = Guarded(C * (T - 1)), Guarded(C * T * 2)
+    if B == 0 and C > 0:
+        with pytest.raises(tdm.TdmError):           # a mean over no samples
+            tdm.seam_discrepancy(band.t, t, seams.t)
+    else:
+        tdm.seam_discrepancy(band.t, t, seams.t)
+    tdm.nonoverlap_drift(band.t, band.t, t, tiles.t, None)
+    tdm.kabsch_stitch(band.t, t, band.t, band.t)
+    tdm.mds_recover(band.t, 0, band.t, band.t)
+    tdm.pairwise_dist(band.t, 0, band.t)
+    tdm.refine_smacof(band.t, 0, band.t, 5, band.t)
+    tdm.scan_nonfinite(band.t)
+    assert tdm.ctx_sync() == 0
+    assert band.intact() and seams.intact() and tiles.intact()

@@ -367,8 +367,8 @@ tdm_status tdm_ddim_step(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, 
     if ((s = check_tiling(ctx, tiling, &t)) != TDM_OK) return s;
     if (step < 0 || step >= sched->S) return fail(ctx, TDM_EINVAL, "step %d outside [0, %d)", step, sched->S);
     if (!std::isfinite(w)) return fail(ctx, TDM_EINVAL, "w is not finite");
+    if (t.n_maps() == 0) return TDM_OK;    // an empty batch is a no-op, whatever its pointers
     if (w != 0.0f && eps_u == nullptr) return fail(ctx, TDM_EINVAL, "eps_u is NULL but w != 0");
-    if (t.n_maps() == 0) return TDM_OK;
     if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, eps_c, "eps_c")) != TDM_OK)
         return s;
     if (w != 0.0f && (s = check_maps(ctx, eps_u, "eps_u")) != TDM_OK) return s;
