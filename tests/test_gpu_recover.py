@@ -110,3 +110,21 @@ def test_recovery_of_sampler_output(tdm):
     Xo, _ = omds.classical_mds(ref)
     e = normwise(host(rec).reshape(-1, 64, 64), omds.pairwise_distances(Xo))
     assert e.max() <= TOL_RECOVER, e.max()
+
+
+def test_mds_rank_deficient_maps(tdm):
+    # points on a plane (lambda_3 = 0) and on a line (lambda_2 = lambda_3 = 0):
+    # the distances rebuild, the null eigenvalues come out ~0, and the
+    # eigen-solve converges without a flag
+    g = np.random.default_rng(3)
+    plane = np.concatenate([g.standard_normal((4, 64, 2)) * 3.0, np.zeros((4, 64, 1))], axis=2)
+    line = np.concatenate([g.standard_normal((4, 64, 1)) * 3.0, np.zeros((4, 64, 2))], axis=2)
+    rot = np.stack([synth.random_orthogonal(g) for _ in range(8)])
+    pts = np.einsum("mij,mnj->mni", rot, np.concatenate([plane, line]))
+    D = synth.exact_distance_maps(pts).astype(np.float32)
+    X, lam, flags = _recover(tdm, D)
+    assert flags == 0 and np.all(np.isfinite(X))
+    e = normwise(omds.pairwise_distances(X), D.astype(np.float64))
+    assert e.max() <= TOL_RECOVER, e.max()
+    assert np.all(np.abs(lam[:4, 2]) <= 1e-5 * lam[:4, 0])
+    assert np.all(np.abs(lam[4:, 1:]) <= 1e-5 * lam[4:, :1])
