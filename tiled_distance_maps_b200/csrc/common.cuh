@@ -4,10 +4,47 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <map>
+#include <mutex>
 
 #include "internal.h"
 
 namespace tdm {
+
+// Launch shape of a kernel on the current device: resident CTAs per SM at the
+// given block size and dynamic shared memory (the shared-memory attribute set
+// when above the default 48 KiB) and the SM count, computed once per
+// (device, kernel) and cached, so launches repeat no driver queries.
+struct LaunchShape {
+    int per_sm, sms;
+};
+
+inline cudaError_t launch_shape(const void *kernel, int threads, size_t smem, LaunchShape *out) {
+    static std::mutex mu;
+    static std::map<std::pair<int, const void *>, LaunchShape> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find({dev, kernel});
+    if (it != cache.end()) {
+        *out = it->second;
+        return cudaSuccess;
+    }
+    if (smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    LaunchShape shape{0, 0};
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&shape.per_sm, kernel, threads, smem);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&shape.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (shape.per_sm < 1) shape.per_sm = 1;
+    cache[{dev, kernel}] = shape;
+    *out = shape;
+    return cudaSuccess;
+}
+
 
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
 // as 1, 2, 3", SC'11): per round, counter words 0 and 2 are multiplied by the

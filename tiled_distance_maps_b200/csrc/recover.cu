@@ -405,14 +405,11 @@ cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigva
     if (n <= 0) return cudaSuccess;
     const size_t smem = sizeof(float) * (size_t)kMdsWarps * (kN * kLd + kN * 4 + kN);
     static_assert((kMdsWarps * kN * kLd * sizeof(float)) % 16 == 0, "float4 alignment of the V tiles");
-    cudaError_t e = cudaFuncSetAttribute(mds_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    LaunchShape shape;
+    const cudaError_t e = launch_shape(reinterpret_cast<const void *>(mds_kernel), kMdsWarps * 32, smem, &shape);
     if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mds_kernel, kMdsWarps * 32, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
     int64_t grid = (n + kMdsWarps - 1) / kMdsWarps;
-    const int64_t cap = (int64_t)sms() * per_sm;
+    const int64_t cap = (int64_t)shape.sms * shape.per_sm;
     if (grid > cap) grid = cap;
     mds_kernel<<<(int)grid, kMdsWarps * 32, smem, st>>>(maps, n, coords, eigvals, flags);
     return cudaGetLastError();

@@ -206,16 +206,11 @@ cudaError_t launch_refine(const float *maps, int64_t n, float *coords, int itera
                           cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
     const size_t smem = sizeof(float) * (size_t)kRefWarps * kRefWarpFloats;
-    cudaError_t e = cudaFuncSetAttribute(refine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    LaunchShape shape;
+    const cudaError_t e = launch_shape(reinterpret_cast<const void *>(refine_kernel), kRefWarps * 32, smem, &shape);
     if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, refine_kernel, kRefWarps * 32, smem);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t grid = (n + kRefWarps - 1) / kRefWarps;
-    const int64_t cap = (int64_t)sms * (per_sm < 1 ? 1 : per_sm);
+    const int64_t cap = (int64_t)shape.sms * shape.per_sm;
     if (grid > cap) grid = cap;
     refine_kernel<<<(int)grid, kRefWarps * 32, smem, st>>>(maps, n, coords, iterations, stress);
     return cudaGetLastError();
