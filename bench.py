@@ -33,6 +33,7 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 WORKLOAD = synth.WORKLOADS["chain32_b1000_cfg"]
+SMALL = synth.WORKLOADS["chain4_b8_s50"]
 METRIC = "map-denoise-steps/sec (64-bead fp32 maps) on 1 B200; % FP32/HBM roofline"
 UNIT = "map-steps/s"
 
@@ -407,6 +408,8 @@ def run_ours(args, rank, world, local_rank):
     flags |= tdm.ctx_sync(ctx)
     del ref_maps
 
+    nx["small_case"] = _small_case(tdm, ctx, dev)
+
     t = torch.tensor([ms, e2e_ms, float(np.mean(run_ms))], device=dev, dtype=torch.float64)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -448,6 +451,7 @@ def run_ours(args, rank, world, local_rank):
                               "note": "one DDIM step of 32,000 maps, CFG w=1: read x, eps_c, eps_u, write x "
                                       "(64 KiB per map); timed separately from the step above"},
             "next_rows": _next_rows(nx, n_maps, B, T, L, peak, float(peaks["hbm_gbs"])),
+            "small_case": nx["small_case"],
             "mds_not_converged": bool(flags & tdm.FLAG_MDS_NOT_CONVERGED),
             "peaks": kind,
         }
@@ -465,6 +469,57 @@ def run_ours(args, rank, world, local_rank):
                                               "float64 numpy"}
         print(json.dumps(line), flush=True)
     return 0
+
+
+def _small_case(tdm, ctx, dev, reps: int = 50) -> dict:
+    """The latency-bound small workload (1 chain x 4 tiles x 8 samples, S = 50,
+    w = 0, s_c = 0.1, projection every step): the whole pipeline per call,
+    launched back to back on the stream and replayed from a CUDA graph.  Each
+    rank measures its own GPU; no collective is captured."""
+    import torch
+    wl = SMALL
+    t = tdm.Tiling(C=1, T=wl.T, B=wl.B, overlap=wl.overlap, sync_every=wl.sync_every)
+    n = t.n_maps
+    sch = tdm.Schedule(wl.S, wl.eta, ctx=ctx)
+    x0 = torch.from_numpy(synth.chain_x0(wl.seed, 1, wl.T, sigma=wl.sigma)).to(dev)
+    maps, coords = torch.empty(n * 4096, device=dev), torch.empty(n * 192, device=dev)
+    rec, disc = torch.empty(n * 4096, device=dev), torch.empty(wl.T - 1, device=dev)
+
+    def pipeline():
+        tdm.ddim_run(sch, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, t, ctx=ctx)
+        tdm.mds_recover(maps, n, coords, ctx=ctx)
+        tdm.pairwise_dist(coords, n, rec, ctx=ctx)
+        tdm.seam_discrepancy(rec, t, disc, ctx=ctx)
+
+    def timed(fn):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(torch.cuda.current_stream())
+        for _ in range(reps):
+            fn()
+        b.record(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e3 / reps
+
+    us_stream = timed(pipeline)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        pipeline()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        pipeline()
+    us_graph = timed(g.replay)
+    del g
+    return {"workload": f"{wl.name}: 1 chain x {wl.T} tiles x {wl.B} samples, DDIM {wl.S} steps, w={wl.w}, "
+                        "MDS + reconstruction + Eq. (6)",
+            "us_per_pipeline_stream": us_stream, "us_per_pipeline_graph": us_graph,
+            "map_steps_per_s_graph": n * wl.S / (us_graph * 1e-6),
+            "note": f"{reps} pipelines back to back; latency-bound, so no roofline"}
 
 
 def _time_flushed(fn, stream, flush, n: int = 10) -> float:
