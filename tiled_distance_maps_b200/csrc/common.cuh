@@ -124,6 +124,37 @@ __device__ __forceinline__ float2 box_muller(uint32_t a, uint32_t b) {
     return make_float2(-r * cs, -r * sn);
 }
 
+// box_muller on the two word pairs (w.x, w.y) and (w.z, w.w) of one Philox
+// call at once, in packed float32 arithmetic (two components per instruction,
+// each rounded as the scalar operation): zc = -(z0, z2) and zs = -(z1, z3),
+// the NEGATED normals of box_muller(w.x, w.y) = (z0, z1) and
+// box_muller(w.z, w.w) = (z2, z3) (negation is exact; the caller folds it
+// into its coefficients).
+__device__ __forceinline__ void box_muller_packed(uint4 w, float2 &zc, float2 &zs) {
+    const float2 f = make_float2(__uint_as_float(0x3F800000u | (w.x >> 9)), __uint_as_float(0x3F800000u | (w.z >> 9)));
+    const float2 fb = make_float2(__uint_as_float(0x3F800000u | (w.y >> 9)), __uint_as_float(0x3F800000u | (w.w >> 9)));
+    const float2 e = __fadd2_rn(f, make_float2(-1.0f, -1.0f));
+    const float2 u1 = __ffma2_rn(f, make_float2(-1.0f, -1.0f), make_float2(2.0f, 2.0f));     // 2 - f, exact product
+    const float2 h = __fadd2_rn(fb, make_float2(-1.5f, -1.5f));
+    float2 lg, r, sn, cs;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg.x) : "f"(u1.x));
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg.y) : "f"(u1.y));
+    const float2 v_log = __fmul2_rn(make_float2(-1.3862943611198906f, -1.3862943611198906f), lg);
+    const float2 v_ser = __fmul2_rn(
+        e, __ffma2_rn(e, __ffma2_rn(e, make_float2(0.6666667f, 0.6666667f), make_float2(1.0f, 1.0f)),
+                      make_float2(2.0f, 2.0f)));
+    const float2 v = make_float2(e.x < 0.015625f ? v_ser.x : v_log.x, e.y < 0.015625f ? v_ser.y : v_log.y);
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r.x) : "f"(v.x));
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r.y) : "f"(v.y));
+    const float2 ang = __fmul2_rn(make_float2(6.2831853071795865f, 6.2831853071795865f), h);
+    asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn.x) : "f"(ang.x));
+    asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs.x) : "f"(ang.x));
+    asm("sin.approx.ftz.f32 %0, %1;" : "=f"(sn.y) : "f"(ang.y));
+    asm("cos.approx.ftz.f32 %0, %1;" : "=f"(cs.y) : "f"(ang.y));
+    zc = __fmul2_rn(r, cs);
+    zs = __fmul2_rn(r, sn);
+}
+
 // The four normals of row quad (r, q): columns 4q .. 4q+3.
 __device__ __forceinline__ float4 quad_normals(int r, int q, uint32_t step_word, uint64_t g, int tag,
                                                const PhiloxKeys &K) {

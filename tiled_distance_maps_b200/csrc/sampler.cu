@@ -210,14 +210,34 @@ __device__ __forceinline__ void lane_normals(const LaneCounter &L, uint32_t step
     }
 }
 
+// The same draws as lane_normals, as negated packed halves (box_muller_packed).
+template <int NS>
+__device__ __forceinline__ void lane_normals_packed(const LaneCounter &L, uint32_t step_word, const int (&tags)[NS],
+                                                    const PhiloxKeys &K, float2 (&zc)[NS], float2 (&zs)[NS]) {
+    const uint64_t p0 = (uint64_t)Philox::M0 * (L.A ^ step_word);
+    const uint32_t w2 = (uint32_t)(p0 >> 32) ^ L.L0 ^ K.k1[1];
+    const uint32_t w3 = (uint32_t)p0;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+        const uint64_t p1 = (uint64_t)Philox::M1 * (L.B ^ ((uint32_t)tags[s] << 24));
+        uint4 c = make_uint4((uint32_t)(p1 >> 32) ^ L.L1 ^ K.k0[1], (uint32_t)p1, w2, w3);
+        c = philox_rounds<2>(c, K);
+        box_muller_packed(c, zc[s], zs[s]);
+    }
+}
+
 template <bool HAS_U, bool HAS_ETA, bool INIT>
 __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
-    extern __shared__ float4 sco[];        // [S] (ka, kx0, kc, ku) then [S] ks
-    float *sks = reinterpret_cast<float *>(sco + a.S);
+    // per step, packed (both halves equal): (ka, kx0) then (-kc, -ku), the noise
+    // coefficients negated for the negated packed normals; then [S] -ks
+    extern __shared__ float4 sco[];
+    float2 *sks = reinterpret_cast<float2 *>(sco + 2 * a.S);
     for (int i = threadIdx.x; i < a.S; i += blockDim.x) {
         const StepCoef c = a.coef[i];
-        sco[i] = make_float4(c.ka, c.kx0, c.kb * a.cc, -(c.kb * a.cu));
-        if (HAS_ETA) sks[i] = c.ks;
+        const float kc = c.kb * a.cc, ku = -(c.kb * a.cu);
+        sco[2 * i] = make_float4(c.ka, c.ka, c.kx0, c.kx0);
+        sco[2 * i + 1] = make_float4(-kc, -kc, -ku, -ku);
+        if (HAS_ETA) sks[i] = make_float2(-c.ks, -c.ks);
     }
     __syncthreads();
 
@@ -234,19 +254,22 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     float *mp = a.maps + (tile * a.B + b) * kMapFloats;
     const uint64_t g = (uint64_t)(a.base + tile * a.B_total + a.b_off + b);
     const float4 xr = ldg4(a.x0 + tile * kMapFloats + r * kN + 4 * q);
+    const float2 r02 = make_float2(xr.x, xr.z), r13 = make_float2(xr.y, xr.w);
     const LaneCounter L = lane_counter(r, q, g, a.K);
 
-    float4 x;
+    // the state as packed column pairs (x0, x2) and (x1, x3) of the quad
+    float2 x02, x13;
     if (INIT) {
         constexpr int kInit[1] = {TDM_STREAM_INIT};
-        float4 z0[1];
-        lane_normals<1>(L, 0u, kInit, a.K, z0);
-        x = z0[0];
+        float2 zc[1], zs[1];
+        lane_normals_packed<1>(L, 0u, kInit, a.K, zc, zs);
+        x02 = __fmul2_rn(zc[0], make_float2(-1.0f, -1.0f));
+        x13 = __fmul2_rn(zs[0], make_float2(-1.0f, -1.0f));
     } else {
-        x = ld4(mp + r * kN + 4 * q);
+        const float4 x = ld4(mp + r * kN + 4 * q);
+        x02 = make_float2(x.x, x.z);
+        x13 = make_float2(x.y, x.w);
     }
-    // only warps that hold seam pairs (lane 0 is paired in every such warp of
-    // the plan) take part in the projection
     const bool warp_pairs = __shfl_sync(0xffffffffu, paired ? 1 : 0, 0) != 0;
     const bool sync_warp = a.T > 1 && a.sync_every > 0 && warp_pairs;
     // the projection follows the steps counted from the start of the whole
@@ -260,47 +283,38 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     for (int s = 0; s < NS; ++s) tags[s] = kTags[s];
 
     for (int i = a.first; i >= a.last; --i) {
-        const float4 cf = sco[i];
-        float4 z[NS];
-        lane_normals<NS>(L, (uint32_t)i, tags, a.K, z);
-        float4 acc;
-        acc.x = fmaf(cf.z, z[0].x, cf.y * xr.x);
-        acc.y = fmaf(cf.z, z[0].y, cf.y * xr.y);
-        acc.z = fmaf(cf.z, z[0].z, cf.y * xr.z);
-        acc.w = fmaf(cf.z, z[0].w, cf.y * xr.w);
+        const float4 c0 = sco[2 * i], c1 = sco[2 * i + 1];
+        const float2 ka = make_float2(c0.x, c0.y), kx0 = make_float2(c0.z, c0.w);
+        const float2 nkc = make_float2(c1.x, c1.y), nku = make_float2(c1.z, c1.w);
+        float2 zc[NS], zs[NS];
+        lane_normals_packed<NS>(L, (uint32_t)i, tags, a.K, zc, zs);
+        float2 a02 = __ffma2_rn(nkc, zc[0], __fmul2_rn(kx0, r02));
+        float2 a13 = __ffma2_rn(nkc, zs[0], __fmul2_rn(kx0, r13));
         if (HAS_U) {
-            acc.x = fmaf(cf.w, z[1].x, acc.x);
-            acc.y = fmaf(cf.w, z[1].y, acc.y);
-            acc.z = fmaf(cf.w, z[1].z, acc.z);
-            acc.w = fmaf(cf.w, z[1].w, acc.w);
+            a02 = __ffma2_rn(nku, zc[1], a02);
+            a13 = __ffma2_rn(nku, zs[1], a13);
         }
         if (HAS_ETA) {
-            const float ks = sks[i];
-            const float4 ze = z[NS - 1];
-            acc.x = fmaf(ks, ze.x, acc.x);
-            acc.y = fmaf(ks, ze.y, acc.y);
-            acc.z = fmaf(ks, ze.z, acc.z);
-            acc.w = fmaf(ks, ze.w, acc.w);
+            const float2 nks = sks[i];
+            a02 = __ffma2_rn(nks, zc[NS - 1], a02);
+            a13 = __ffma2_rn(nks, zs[NS - 1], a13);
         }
-        x.x = fmaf(cf.x, x.x, acc.x);
-        x.y = fmaf(cf.x, x.y, acc.y);
-        x.z = fmaf(cf.x, x.z, acc.z);
-        x.w = fmaf(cf.x, x.w, acc.w);
+        x02 = __ffma2_rn(ka, x02, a02);
+        x13 = __ffma2_rn(ka, x13, a13);
         if (sync_warp && --until_sync == 0) {
             until_sync = a.sync_every;
-            float4 o;
-            o.x = __shfl_xor_sync(0xffffffffu, x.x, 16);
-            o.y = __shfl_xor_sync(0xffffffffu, x.y, 16);
-            o.z = __shfl_xor_sync(0xffffffffu, x.z, 16);
-            o.w = __shfl_xor_sync(0xffffffffu, x.w, 16);
+            float2 o02, o13;
+            o02.x = __shfl_xor_sync(0xffffffffu, x02.x, 16);
+            o02.y = __shfl_xor_sync(0xffffffffu, x02.y, 16);
+            o13.x = __shfl_xor_sync(0xffffffffu, x13.x, 16);
+            o13.y = __shfl_xor_sync(0xffffffffu, x13.y, 16);
             if (paired) {
-                x.x = 0.5f * (x.x + o.x);
-                x.y = 0.5f * (x.y + o.y);
-                x.z = 0.5f * (x.z + o.z);
-                x.w = 0.5f * (x.w + o.w);
+                x02 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x02, o02));
+                x13 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x13, o13));
             }
         }
     }
+    const float4 x = make_float4(x02.x, x13.x, x02.y, x13.y);
 
     // unfold: the quad's upper entries go to (r, j) and their mirrors to (j, r)
     if (4 * q > r) {
@@ -451,7 +465,7 @@ cudaError_t launch_ddim_run(const StepCoef *coef, int S, int first, int n_steps,
     const int64_t grid64 = (a.total_warps + 7) / 8;
     if (grid64 > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
     const int grid = (int)grid64;
-    const size_t smem = (size_t)S * (sizeof(float4) + (has_eta ? sizeof(float) : 0));
+    const size_t smem = (size_t)S * (2 * sizeof(float4) + (has_eta ? sizeof(float2) : 0));
     const bool has_u = w != 0.0f;
     if (has_u) {
         if (has_eta) return init_noise ? run_variant<true, true, true>(a, grid, smem, st)
