@@ -59,3 +59,37 @@ def test_null_context_is_rejected_before_any_cuda_call(lib):
     assert lib.tdm_ddim_run(None, None, None, None, ctypes.c_float(0), ctypes.c_float(0), ctypes.c_float(0),
                             ctypes.c_uint64(0), 1, None, None) == 1
     assert lib.tdm_mds_recover(None, None, ctypes.c_int64(0), None, None, None) == 1
+
+
+C_PROG = r"""
+#include <stdio.h>
+#include <string.h>
+#include "tdm.h"
+int main(void) {
+    /* host-only calls: status strings, argument checks, the cosine table */
+    double ab[4];
+    if (strcmp(tdm_status_str(TDM_OK), "ok") != 0) return 1;
+    if (tdm_ddim_run(NULL, NULL, NULL, NULL, 0.f, 0.f, 0.f, 0u, 1, NULL, NULL) != TDM_EINVAL) return 2;
+    if (tdm_cosine_alphas_bar(4, 0.008, ab) != TDM_OK) return 3;
+    if (!(ab[0] < 1.0 && ab[3] < ab[2] && ab[3] > 0.0)) return 4;
+    if (tdm_cosine_alphas_bar(0, 0.008, ab) != TDM_EINVAL) return 5;
+    printf("%.17g\n", ab[1]);
+    return 0;
+}
+"""
+
+
+def test_header_is_c99_and_links_from_c(tmp_path):
+    # the boundary is plain C: the header compiles as strict C99 and a C
+    # program links against the library and calls its host entry points
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROG)
+    exe = tmp_path / "abi"
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(LIB)
+    subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                    "-L", libdir, "-ltdm", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out
+    from oracle.schedule import cosine_alphas_bar
+    assert abs(float(out.stdout) - cosine_alphas_bar(4, 0.008)[1]) <= 1e-15
