@@ -96,30 +96,40 @@ __global__ void __launch_bounds__(256) seam_finalize_kernel(const float *__restr
     }
 }
 
-// One warp per seam, all samples: out[seam] directly (few samples per seam).
+// One CTA per seam, all samples: out[seam] directly (few samples per seam).
+// Thread e sums entry e of the block difference over the samples (unrolled,
+// so the loads of several samples are in flight together); the CTA then
+// reduces |mean| over the entries in a fixed order.
 __global__ void __launch_bounds__(256) seam_direct_kernel(const float *__restrict__ maps, int64_t n_seams,
                                                           int T, int B, int o, float inv_b,
                                                           float *__restrict__ out) {
-    const int lane = threadIdx.x & 31;
+    __shared__ float red[8];
     const int s = kN - o;
     const int oo = o * o;
-    for (int64_t seam = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; seam < n_seams;
-         seam += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int64_t seam = blockIdx.x; seam < n_seams; seam += gridDim.x) {
         const int64_t c = seam / (T - 1);
         const int k = (int)(seam - c * (T - 1));
         const float *ta = maps + ((c * T + k) * B) * kMapFloats;
         const float *tb = maps + ((c * T + k + 1) * B) * kMapFloats;
         float local = 0.0f;
-        for (int e = lane; e < oo; e += 32) {
+        for (int e = threadIdx.x; e < oo; e += blockDim.x) {
             const int i = e / o, j = e - (e / o) * o;
-            const int offa = (s + i) * kN + (s + j), offb = i * kN + j;
+            const float *pa = ta + (s + i) * kN + (s + j), *pb = tb + i * kN + j;
             float acc = 0.0f;
-            for (int b = 0; b < B; ++b)
-                acc += __ldg(ta + (int64_t)b * kMapFloats + offa) - __ldg(tb + (int64_t)b * kMapFloats + offb);
+#pragma unroll 8
+            for (int b = 0; b < B; ++b) acc += __ldg(pa + (int64_t)b * kMapFloats) - __ldg(pb + (int64_t)b * kMapFloats);
             local += fabsf(acc * inv_b);
         }
         local = warp_sum(local);
-        if (lane == 0) out[seam] = local / (float)oo;
+        if (lane == 0) red[warp] = local;
+        __syncthreads();
+        if (warp == 0) {
+            float v = lane < nwarps ? red[lane] : 0.0f;
+            v = warp_sum(v);
+            if (lane == 0) out[seam] = v / (float)oo;
+        }
+        __syncthreads();
     }
 }
 
@@ -180,10 +190,12 @@ cudaError_t launch_seam_finalize(const float *src, const Tiling &t, int chunks, 
     const int64_t n_seams = (int64_t)t.C * (t.T - 1);
     if (n_seams <= 0) return cudaSuccess;
     if (chunks == 0) {
-        int64_t grid = (n_seams * 32 + 255) / 256;
-        const int64_t cap = (int64_t)sm_count() * 16;
+        const int oo = t.overlap * t.overlap;
+        const int threads = oo >= 256 ? 256 : ((oo + 31) / 32) * 32;
+        int64_t grid = n_seams;
+        const int64_t cap = (int64_t)sm_count() * 32;
         if (grid > cap) grid = cap;
-        seam_direct_kernel<<<(int)grid, 256, 0, st>>>(src, n_seams, t.T, t.B, t.overlap, (float)inv_b, out);
+        seam_direct_kernel<<<(int)grid, threads, 0, st>>>(src, n_seams, t.T, t.B, t.overlap, (float)inv_b, out);
     } else {
         if (n_seams > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
         seam_finalize_kernel<<<(unsigned)n_seams, 256, 0, st>>>(src, t.overlap * t.overlap, chunks,
