@@ -204,11 +204,27 @@ def init_schedule(S: int, eta: float = 0.0, **kw) -> Schedule:
     return Schedule(S, eta, **kw)
 
 
+_torch = None
+_raw_stream = None
+
+
+def _t():
+    """torch, imported on first use (the package imports without it)."""
+    global _torch, _raw_stream
+    if _torch is None:
+        import torch
+        _torch = torch
+        # the current stream's handle without building a Stream object; the
+        # public call is the fallback
+        _raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    return _torch
+
+
 def _ptr(t, name: str, ctx: Context | None = None):
     """Device pointer of a CUDA float32 contiguous tensor (None -> NULL)."""
     if t is None:
         return None
-    import torch
+    torch = _t()
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
@@ -217,13 +233,15 @@ def _ptr(t, name: str, ctx: Context | None = None):
         raise ValueError(f"{name} must be float32, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if ctx is not None and t.device.index != ctx.device:
-        raise ValueError(f"{name} is on cuda:{t.device.index}, context on cuda:{ctx.device}")
+    if ctx is not None and t.get_device() != ctx.device:
+        raise ValueError(f"{name} is on cuda:{t.get_device()}, context on cuda:{ctx.device}")
     return _vp(t.data_ptr())
 
 
 def _stream(ctx: Context):
-    import torch
+    torch = _t()
+    if _raw_stream is not None:
+        return _vp(_raw_stream(ctx.device))
     return _vp(torch.cuda.current_stream(ctx.device).cuda_stream)
 
 
