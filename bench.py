@@ -263,11 +263,10 @@ def run_ours(args, rank, world, local_rank):
         tdm.ddim_run(sched, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, tiling, ctx=ctx)
         if i_timed is not None:
             ev_run[2 * i_timed + 1].record(stream)
-        tdm.mds_recover(maps, n_maps, coords, eig, ctx=ctx)
-        tdm.pairwise_dist(coords, n_maps, rec, ctx=ctx)
+        tdm.mds_reconstruct(maps, n_maps, coords, rec, eig, ctx=ctx)
         sharded_seam_discrepancy(rec, tiling, sums, disc, ctx=ctx)
 
-    launches_per_step = 1 + 1 + 1 + (2 if _seam_chunks(T - 1, B) > 1 else 1) + 1
+    launches_per_step = 1 + 1 + (2 if _seam_chunks(T - 1, B) > 1 else 1) + 1
 
     def barrier():
         if world > 1:
@@ -305,8 +304,7 @@ def run_ours(args, rank, world, local_rank):
 
     def step_into(cb, eb, db):
         tdm.ddim_run(sched, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, tiling, ctx=ctx)
-        tdm.mds_recover(maps, n_maps, cb, eb, ctx=ctx)
-        tdm.pairwise_dist(cb, n_maps, rec, ctx=ctx)
+        tdm.mds_reconstruct(maps, n_maps, cb, rec, eb, ctx=ctx)
         sharded_seam_discrepancy(rec, tiling, sums, db, ctx=ctx)
 
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -487,8 +485,7 @@ def _small_case(tdm, ctx, dev, reps: int = 50) -> dict:
 
     def pipeline():
         tdm.ddim_run(sch, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, t, ctx=ctx)
-        tdm.mds_recover(maps, n, coords, ctx=ctx)
-        tdm.pairwise_dist(coords, n, rec, ctx=ctx)
+        tdm.mds_reconstruct(maps, n, coords, rec, ctx=ctx)
         tdm.seam_discrepancy(rec, t, disc, ctx=ctx)
 
     def timed(fn):

@@ -274,6 +274,14 @@ tdm_status tdm_box_muller(tdm_ctx *ctx, const uint32_t *words, int64_t n_pairs, 
 tdm_status tdm_mds_recover(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords,
                            float *eigvals_opt, tdm_stream stream);
 
+/* tdm_mds_recover and tdm_pairwise_dist of its coordinates in one pass: the
+ * same coordinates, eigenvalues and flags, and dist_out (device
+ * [n_maps][64][64], caller-owned, 16-byte aligned) equal to what
+ * tdm_pairwise_dist writes for them, bit for bit, without reading the
+ * coordinates back from memory. */
+tdm_status tdm_mds_reconstruct(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, float *eigvals_opt,
+                               float *dist_out, tdm_stream stream);
+
 /* maps_out[m][i][j] = || coords[m][i] - coords[m][j] ||_2 (device; zero diagonal). */
 tdm_status tdm_pairwise_dist(tdm_ctx *ctx, const float *coords, int64_t n_maps, float *maps_out,
                              tdm_stream stream);

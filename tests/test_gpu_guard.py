@@ -90,6 +90,9 @@ def test_recovery_outputs_stay_in_bounds(tdm, n):
     stress = Guarded(n)
     tdm.refine_smacof(maps, n, coords.t, 3, stress.t)
     assert coords.intact() and stress.intact(), "refine_smacof"
+    dist = Guarded(n * 4096)
+    tdm.mds_reconstruct(maps, n, coords.t, dist.t, eig.t)
+    assert coords.intact() and eig.intact() and dist.intact(), "mds_reconstruct"
 
 
 @pytest.mark.parametrize("C,T,B,o", [(2, 3, 5, 12), (1, 1, 2, 12), (1, 4, 3, 7)])
@@ -154,6 +157,7 @@ def test_empty_inputs_write_nothing(tdm, C, T, B):
     tdm.nonoverlap_drift(band.t, band.t, t, tiles.t, None)
     tdm.kabsch_stitch(band.t, t, band.t, band.t)
     tdm.mds_recover(band.t, 0, band.t, band.t)
+    tdm.mds_reconstruct(band.t, 0, band.t, band.t, band.t)
     tdm.pairwise_dist(band.t, 0, band.t)
     tdm.refine_smacof(band.t, 0, band.t, 5, band.t)
     tdm.scan_nonfinite(band.t)

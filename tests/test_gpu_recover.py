@@ -128,3 +128,18 @@ def test_mds_rank_deficient_maps(tdm):
     assert e.max() <= TOL_RECOVER, e.max()
     assert np.all(np.abs(lam[:4, 2]) <= 1e-5 * lam[:4, 0])
     assert np.all(np.abs(lam[4:, 1:]) <= 1e-5 * lam[4:, :1])
+
+
+@pytest.mark.parametrize("n", [1, 37, 1000])
+def test_fused_reconstruction_equals_the_two_calls(tdm, n):
+    # tdm_mds_reconstruct writes the coordinates, eigenvalues and distance
+    # maps that tdm_mds_recover followed by tdm_pairwise_dist write, bit for bit
+    maps = dev(synth.cloud_maps(2, 0, n)).reshape(-1)
+    c1, e1, d1 = (torch.empty(n * k, device="cuda") for k in (192, 3, 4096))
+    c2, e2, d2 = (torch.empty(n * k, device="cuda") for k in (192, 3, 4096))
+    tdm.mds_recover(maps, n, c1, e1)
+    tdm.pairwise_dist(c1, n, d1)
+    tdm.mds_reconstruct(maps, n, c2, d2, e2)
+    assert tdm.ctx_sync() == 0
+    for a, b in ((c1, c2), (e1, e2), (d1, d2)):
+        np.testing.assert_array_equal(host(a), host(b))

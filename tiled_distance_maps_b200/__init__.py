@@ -69,6 +69,7 @@ _SIGS = {
     "tdm_nonoverlap_drift": (_i32, [_vp, _vp, _vp, _P(CTiling), _vp, _vp, _vp]),
     "tdm_cosine_alphas_bar": (_i32, [_i32, _f64, _vp]),
     "tdm_scan_nonfinite": (_i32, [_vp, _vp, _i64, _vp]),
+    "tdm_mds_reconstruct": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -319,6 +320,19 @@ def mds_recover(maps, n_maps: int, coords, eigvals=None, ctx: Context | None = N
     ctx.check(_lib.tdm_mds_recover(ctx.handle, _ptr(maps, "maps", ctx), int(n_maps), _ptr(coords, "coords", ctx),
                                    _ptr(eigvals, "eigvals", ctx), _stream(ctx)))
     return coords
+
+
+def mds_reconstruct(maps, n_maps: int, coords, dist_out, eigvals=None, ctx: Context | None = None):
+    """MDS recovery and the distance maps of its coordinates in one pass (see
+    tdm_mds_reconstruct)."""
+    ctx = ctx or context(maps.device.index)
+    _need(maps, n_maps * 4096, "maps")
+    _need(coords, n_maps * 192, "coords")
+    _need(dist_out, n_maps * 4096, "dist_out")
+    _need(eigvals, n_maps * 3, "eigvals")
+    ctx.check(_lib.tdm_mds_reconstruct(ctx.handle, _ptr(maps, "maps", ctx), int(n_maps), _ptr(coords, "coords", ctx),
+                                       _ptr(eigvals, "eigvals", ctx), _ptr(dist_out, "dist_out", ctx), _stream(ctx)))
+    return dist_out
 
 
 def pairwise_dist(coords, n_maps: int, maps_out, ctx: Context | None = None):

@@ -521,7 +521,26 @@ tdm_status tdm_mds_recover(tdm_ctx *ctx, const float *maps, int64_t n_maps, floa
     if (eigvals_opt != nullptr && (reinterpret_cast<uintptr_t>(eigvals_opt) & 3u))
         return fail(ctx, TDM_EINVAL, "eigvals is not 4-byte aligned");
     DeviceScope ds(ctx->device);
-    cudaError_t e = tdm::launch_mds(maps, n_maps, coords, eigvals_opt, ctx->d_flags, static_cast<cudaStream_t>(stream));
+    cudaError_t e = tdm::launch_mds(maps, n_maps, coords, eigvals_opt, ctx->d_flags, nullptr,
+                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "mds launch");
+}
+
+tdm_status tdm_mds_reconstruct(tdm_ctx *ctx, const float *maps, int64_t n_maps, float *coords, float *eigvals_opt,
+                               float *dist_out, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_mds_reconstruct");
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (n_maps < 0) return fail(ctx, TDM_EINVAL, "n_maps < 0");
+    if (n_maps == 0) return TDM_OK;
+    tdm_status s;
+    if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, coords, "coords")) != TDM_OK ||
+        (s = check_maps(ctx, dist_out, "dist_out")) != TDM_OK)
+        return s;
+    if (eigvals_opt != nullptr && (reinterpret_cast<uintptr_t>(eigvals_opt) & 3u))
+        return fail(ctx, TDM_EINVAL, "eigvals is not 4-byte aligned");
+    DeviceScope ds(ctx->device);
+    cudaError_t e = tdm::launch_mds(maps, n_maps, coords, eigvals_opt, ctx->d_flags, dist_out,
+                                    static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "mds launch");
 }
 

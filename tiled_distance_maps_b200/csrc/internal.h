@@ -74,7 +74,7 @@ cudaError_t launch_seam_reduce(const float *partial, const Tiling &t, int chunks
                                cudaStream_t st);
 cudaError_t launch_seam_finalize(const float *sums, const Tiling &t, int chunks, double inv_b,
                                  float *out, cudaStream_t st);
-cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigvals, uint32_t *flags,
+cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigvals, uint32_t *flags, float *dist,
                        cudaStream_t st);
 cudaError_t launch_pdist(const float *coords, int64_t n, float *maps, cudaStream_t st);
 cudaError_t launch_refine(const float *maps, int64_t n, float *coords, int iterations, float *stress,

@@ -143,10 +143,18 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i) {
     }
 }
 
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+template <bool DIST>
 __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__restrict__ maps, int64_t n,
                                                                 float *__restrict__ coords,
                                                                 float *__restrict__ eig,
-                                                                uint32_t *__restrict__ flags) {
+                                                                uint32_t *__restrict__ flags,
+                                                                float *__restrict__ dist) {
     extern __shared__ __align__(16) float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float *sD = smem + warp * (kN * kLd);
@@ -341,6 +349,33 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
             X[i1 * 3 + c] = u1[c] * sq;
         }
         if (eig != nullptr && lane < 3) eig[m * 3 + lane] = (lane == 0 ? th[0] : lane == 1 ? th[1] : th[2]) * inv_scale;
+        if (DIST) {
+            // the distance map of the coordinates, as pdist_kernel computes it:
+            // the coordinates go to shared memory (the V arrays are free now),
+            // then row r is written by the whole warp, two columns per lane,
+            // with coalesced 8-byte streaming stores
+            float *sc = reinterpret_cast<float *>(sV01);    // x[64], y[64], z[64]
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < kK; ++c) {
+                const float sq = sqrtf(fmaxf(th[c], 0.0f) * inv_scale);
+                sc[c * kN + i0] = u0[c] * sq;
+                sc[c * kN + i1] = u1[c] * sq;
+            }
+            __syncwarp();
+            const float2 cx = reinterpret_cast<const float2 *>(sc)[lane];
+            const float2 cy = reinterpret_cast<const float2 *>(sc + kN)[lane];
+            const float2 cz = reinterpret_cast<const float2 *>(sc + 2 * kN)[lane];
+            float2 *out = reinterpret_cast<float2 *>(dist + m * kMapFloats) + lane;
+#pragma unroll 4
+            for (int row = 0; row < kN; ++row) {
+                const float xi = sc[row], yi = sc[kN + row], zi = sc[2 * kN + row];
+                float2 d;
+                d.x = sqrt_approx(fmaf(zi - cz.x, zi - cz.x, fmaf(yi - cy.x, yi - cy.x, (xi - cx.x) * (xi - cx.x))));
+                d.y = sqrt_approx(fmaf(zi - cz.y, zi - cz.y, fmaf(yi - cy.y, yi - cy.y, (xi - cx.y) * (xi - cx.y))));
+                __stcs(out + row * (kN / 2), d);
+            }
+        }
         __syncwarp();
     }
 }
@@ -353,11 +388,6 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
 // diagonal).
 constexpr int kPdistMaps = 4;
 
-__device__ __forceinline__ float sqrt_approx(float x) {
-    float r;
-    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
 
 __global__ void __launch_bounds__(256) pdist_kernel(const float *__restrict__ coords, int64_t n,
                                                     float *__restrict__ maps) {
@@ -400,18 +430,23 @@ int sms() {
 
 }  // namespace
 
-cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigvals, uint32_t *flags,
+cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigvals, uint32_t *flags, float *dist,
                        cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
     const size_t smem = sizeof(float) * (size_t)kMdsWarps * (kN * kLd + kN * 4 + kN);
     static_assert((kMdsWarps * kN * kLd * sizeof(float)) % 16 == 0, "float4 alignment of the V tiles");
+    const void *kern = dist != nullptr ? reinterpret_cast<const void *>(mds_kernel<true>)
+                                       : reinterpret_cast<const void *>(mds_kernel<false>);
     LaunchShape shape;
-    const cudaError_t e = launch_shape(reinterpret_cast<const void *>(mds_kernel), kMdsWarps * 32, smem, &shape);
+    const cudaError_t e = launch_shape(kern, kMdsWarps * 32, smem, &shape);
     if (e != cudaSuccess) return e;
     int64_t grid = (n + kMdsWarps - 1) / kMdsWarps;
     const int64_t cap = (int64_t)shape.sms * shape.per_sm;
     if (grid > cap) grid = cap;
-    mds_kernel<<<(int)grid, kMdsWarps * 32, smem, st>>>(maps, n, coords, eigvals, flags);
+    if (dist != nullptr)
+        mds_kernel<true><<<(int)grid, kMdsWarps * 32, smem, st>>>(maps, n, coords, eigvals, flags, dist);
+    else
+        mds_kernel<false><<<(int)grid, kMdsWarps * 32, smem, st>>>(maps, n, coords, eigvals, flags, nullptr);
     return cudaGetLastError();
 }
 
