@@ -9,7 +9,12 @@
  * (the distance-geometry initialisation of §3.1), pairwise-distance
  * reconstruction and the seam discrepancy of §5.5 Eq. (6).  The trained U-Net
  * is replaced by a stand-in noise predictor: the ideal denoiser toward a known
- * x0 plus counter-based Philox noise.
+ * x0 plus counter-based Philox noise.  Beside that path: SMACOF coordinate
+ * refinement (§3.1), Kabsch stitching of tiles into chains with the per-seam
+ * residual (§4.3.2, §5.5 Fig. 4), the non-overlap drift of the
+ * synchronisation-frequency sweep (§5.7 Table 8), resumable parts of a run, the
+ * cosine schedule of the caller-table path, the noise primitives and a
+ * NaN/inf scan.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
