@@ -55,3 +55,21 @@ def test_random_fused_runs(tdm, k):
                 B_total, overlap=o, sync_every=c["K"], sample_id_base=c["base"], x_T=x_T)
     got = host(maps).reshape(C, T, B, 64, 64)
     assert_maps_close(got, ref, TOL_MAP, f"config {c}")
+
+
+@pytest.mark.parametrize("k", range(24))
+def test_random_per_step_runs(tdm, k):
+    # the per-step path (stand-in eps, DDIM step, projection when due), which
+    # also takes overlaps that are not a multiple of 4
+    from tests.test_gpu_sampler import _gpu_per_step
+    g = np.random.default_rng([4048, k])
+    C, T, B = int(g.integers(1, 3)), int(g.integers(1, 5)), int(g.integers(1, 4))
+    o = int(g.integers(1, 33))
+    K, S = int(g.choice([0, 1, 2, 3])), int(g.choice([1, 2, 4, 5, 8, 10]))
+    eta, w = float(g.choice([0.0, 1.0])), float(g.choice([0.0, 1.0, 2.0]))
+    seed = int(g.integers(0, 2 ** 40))
+    t = tdm.Tiling(C=C, T=T, B=B, overlap=o, sync_every=K)
+    x0 = synth.chain_x0(k, C, T, overlap=o)
+    got = _gpu_per_step(tdm, tdm.Schedule(S, eta=eta), x0, t, w, 0.1, 0.3, seed)[-1]
+    ref = o_run(x0, osched.Schedule(S=S, eta=eta), w, 0.1, 0.3, seed, np.arange(B), B, overlap=o, sync_every=K)
+    assert_maps_close(got, ref, TOL_MAP, f"per-step C={C} T={T} B={B} o={o} K={K} S={S} eta={eta} w={w}")
