@@ -580,6 +580,150 @@ def _seam_chunks(n_seams, B):
     return max(1, min(ch, -(-B // 8)))
 
 
+def _events_ms(fn, reps: int = 1) -> float:
+    """Device ms of ``reps`` back-to-back calls of ``fn`` (one untimed first)."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_configs(args) -> int:
+    """One JSON line per workload (not the bench contract line): throughput of
+    the path on each of the five workloads, on one GPU, with the oracle timed
+    beside the ones it can sample.  Inputs of the 1,000,000-map recovery are
+    drawn on the device by torch (timing only; parity is the tests' job)."""
+    import torch
+    import tiled_distance_maps_b200 as tdm
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ctx = tdm.context(0)
+    peaks, _ = measured_peaks()
+    alu_peak = alu_peak_ops(148, float(peaks.get("sm_max_mhz", 1965.0)) / 1e3)
+    lines = []
+
+    # cfg1: the small pipeline (latency)
+    sc = _small_case(tdm, ctx, dev)
+    wl = SMALL
+    t0 = time.perf_counter()
+    oracle_small(wl)
+    dt = time.perf_counter() - t0
+    lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
+                  "value": sc["map_steps_per_s_graph"], "us_per_pipeline_graph": sc["us_per_pipeline_graph"],
+                  "us_per_pipeline_stream": sc["us_per_pipeline_stream"],
+                  "oracle_map_steps_per_s_1core": wl.n_maps * wl.S / dt, "bound": "latency"})
+
+    # cfg2: the headline step (fused run + MDS with reconstruction + Eq. 6)
+    wl = WORKLOAD
+    t = tdm.Tiling(C=1, T=wl.T, B=wl.B, overlap=wl.overlap, sync_every=wl.sync_every)
+    n = t.n_maps
+    sch = tdm.Schedule(wl.S, wl.eta, ctx=ctx)
+    x0 = torch.from_numpy(synth.chain_x0(wl.seed, 1, wl.T, sigma=wl.sigma)).to(dev)
+    maps, coords, rec = (torch.empty(n * k, device=dev) for k in (4096, 192, 4096))
+    disc = torch.empty(wl.T - 1, device=dev)
+
+    def step2():
+        tdm.ddim_run(sch, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, t, ctx=ctx)
+        tdm.mds_reconstruct(maps, n, coords, rec, ctx=ctx)
+        tdm.seam_discrepancy(rec, t, disc, ctx=ctx)
+    ms = _events_ms(step2, 5)
+    lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
+                  "value": n * wl.S / (ms / 1e3), "ms_per_step": ms, "bound": "alu (fused run)"})
+    del maps, coords, rec
+
+    # cfg3: the step sweep on the 32-tile x 100-sample chain, w = 0
+    wl = synth.WORKLOADS["chain32_b100_sweep"]
+    t = tdm.Tiling(C=1, T=wl.T, B=wl.B, overlap=wl.overlap, sync_every=wl.sync_every)
+    n = t.n_maps
+    x0 = torch.from_numpy(synth.chain_x0(wl.seed, 1, wl.T)).to(dev)
+    maps = torch.empty(n * 4096, device=dev)
+    sweep = []
+    for eta in wl.extra["eta"]:
+        for S in wl.extra["S"]:
+            sch = tdm.Schedule(S, eta, ctx=ctx)
+            ms = _events_ms(lambda: tdm.ddim_run(sch, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, t, ctx=ctx), 3)
+            ns = 1 + (1 if eta > 0 else 0)
+            ops = ops_per_map_step(ns) * n * S + QUADS_PER_MAP * n * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR)
+            sweep.append({"S": S, "eta": eta, "ms": ms, "map_steps_per_s": n * S / (ms / 1e3),
+                          "alu_frac": ops / (ms / 1e3) / alu_peak})
+    lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
+                  "value": sum(x["map_steps_per_s"] for x in sweep) / len(sweep), "runs": sweep,
+                  "note": "value: mean over the 10 runs; alu_frac against the derived lane-op peak"})
+    del maps
+
+    # cfg4: 2658 regions x {w=0, w=1} x 256 samples, untiled, in chunks of 2^16 maps
+    wl = synth.WORKLOADS["genome2658_b256_untiled"]
+    R, B, S = wl.C, wl.B, wl.S
+    chunk_regions = wl.extra["chunk_maps"] // B
+    sch = tdm.Schedule(S, ctx=ctx)
+    maps = torch.empty(chunk_regions * B * 4096, device=dev)
+    total_ms, total_ops = 0.0, 0
+    for gi, w in enumerate(wl.extra["w"]):
+        for r0 in range(0, R, chunk_regions):
+            nr = min(chunk_regions, R - r0)
+            x0 = torch.from_numpy(synth.region_x0(wl.seed, np.arange(r0, r0 + nr))).to(dev)
+            tt = tdm.Tiling(C=nr, T=1, B=B, overlap=0, sync_every=0, sample_id_base=gi * R * B + r0 * B)
+            total_ms += _events_ms(lambda: tdm.ddim_run(sch, maps, x0, w, wl.s_c, wl.s_u, wl.seed, tt, ctx=ctx))
+            ns = 1 + (1 if w != 0 else 0)
+            total_ops += ops_per_map_step(ns) * nr * B * S + QUADS_PER_MAP * nr * B * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR)
+    steps4 = 2 * R * B * S
+    lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
+                  "value": steps4 / (total_ms / 1e3), "device_ms": total_ms,
+                  "alu_frac": total_ops / (total_ms / 1e3) / alu_peak,
+                  "note": "1,360,896 trajectories in 22 chunks; the fused runs' device time summed"})
+    del maps
+
+    # cfg5: 1,000,000 noisy point-cloud maps: MDS + reconstruction, Eq. (6) over 31,250 x 32
+    n = 1_000_000
+    maps5 = torch.empty(n * 4096, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    for m0 in range(0, n, 100_000):
+        k = min(100_000, n - m0)
+        sig = torch.rand(k, 1, 1, device=dev, generator=g) * 9.0 + 1.0
+        pts = torch.randn(k, 64, 3, device=dev, generator=g) * sig
+        d = torch.cdist(pts, pts)
+        z = torch.triu(torch.randn(k, 64, 64, device=dev, generator=g), 1)
+        maps5[m0 * 4096:(m0 + k) * 4096] = (d * (1.0 + 0.01 * (z + z.transpose(1, 2)))).reshape(-1)
+        del sig, pts, d, z
+    coords5, rec5 = torch.empty(n * 192, device=dev), torch.empty(n * 4096, device=dev)
+    t5 = tdm.Tiling(C=31250, T=32, B=1, overlap=12, sync_every=0)
+    disc5 = torch.empty(31250 * 31, device=dev)
+    ms_mds = _events_ms(lambda: tdm.mds_reconstruct(maps5, n, coords5, rec5, ctx=ctx))
+    ms_seam = _events_ms(lambda: tdm.seam_discrepancy(rec5, t5, disc5, ctx=ctx))
+    flags = tdm.ctx_sync(ctx)
+    from oracle import mds as omds
+    sample = maps5[:16 * 4096].view(16, 64, 64).cpu().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    Xo, _ = omds.classical_mds(sample)
+    omds.pairwise_distances(Xo)
+    dt = time.perf_counter() - t0
+    lines.append({"config": "recovery_1m", "metric": "maps/sec", "unit": "maps/s",
+                  "value": n / ((ms_mds + ms_seam) / 1e3), "mds_reconstruct_ms": ms_mds, "seam_ms": ms_seam,
+                  "hbm_frac_mds_reconstruct": n * (2 * 16384 + 768) / (ms_mds / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
+                  "oracle_maps_per_s_1core": 16 / dt, "mds_not_converged": bool(flags & tdm.FLAG_MDS_NOT_CONVERGED),
+                  "note": "inputs drawn on the device by torch for timing only"})
+    for line in lines:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def oracle_small(wl):
+    """The oracle's whole small pipeline: fused-run equivalent, MDS, reconstruction, Eq. (6)."""
+    from oracle import mds as omds, schedule as osched, seam as oseam
+    from oracle.ddim import ddim_run
+    x0 = synth.chain_x0(wl.seed, 1, wl.T)
+    out = ddim_run(x0, osched.Schedule(S=wl.S, eta=wl.eta), wl.w, wl.s_c, wl.s_u, wl.seed, np.arange(wl.B), wl.B)
+    X, _ = omds.classical_mds(out.reshape(-1, 64, 64))
+    oseam.seam_discrepancy(omds.pairwise_distances(X).reshape(out.shape))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -587,6 +731,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--configs", action="store_true",
+                    help="one line per workload (throughput of all five) instead of the bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -595,6 +741,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.configs:
+        if world > 1:
+            return 0 if rank else run_configs(args)
+        return run_configs(args)
     if world > 1:
         import datetime
         import torch
