@@ -96,6 +96,33 @@ __global__ void __launch_bounds__(256) seam_finalize_kernel(const float *__restr
     }
 }
 
+// One warp per seam, all samples: out[seam] directly, for many seams with few
+// samples each (lane e sums entry e, e+32, .. over the samples).
+__global__ void __launch_bounds__(256) seam_direct_warp_kernel(const float *__restrict__ maps, int64_t n_seams,
+                                                               int T, int B, int o, float inv_b,
+                                                               float *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int s = kN - o;
+    const int oo = o * o;
+    for (int64_t seam = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; seam < n_seams;
+         seam += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        const int64_t c = seam / (T - 1);
+        const int k = (int)(seam - c * (T - 1));
+        const float *ta = maps + ((c * T + k) * B) * kMapFloats;
+        const float *tb = maps + ((c * T + k + 1) * B) * kMapFloats;
+        float local = 0.0f;
+        for (int e = lane; e < oo; e += 32) {
+            const int i = e / o, j = e - (e / o) * o;
+            const float *pa = ta + (s + i) * kN + (s + j), *pb = tb + i * kN + j;
+            float acc = 0.0f;
+            for (int b = 0; b < B; ++b) acc += __ldg(pa + (int64_t)b * kMapFloats) - __ldg(pb + (int64_t)b * kMapFloats);
+            local += fabsf(acc * inv_b);
+        }
+        local = warp_sum(local);
+        if (lane == 0) out[seam] = local / (float)oo;
+    }
+}
+
 // One CTA per seam, all samples: out[seam] directly (few samples per seam).
 // Thread e sums entry e of the block difference over the samples (unrolled,
 // so the loads of several samples are in flight together); the CTA then
@@ -190,12 +217,20 @@ cudaError_t launch_seam_finalize(const float *src, const Tiling &t, int chunks, 
     const int64_t n_seams = (int64_t)t.C * (t.T - 1);
     if (n_seams <= 0) return cudaSuccess;
     if (chunks == 0) {
-        const int oo = t.overlap * t.overlap;
-        const int threads = oo >= 256 ? 256 : ((oo + 31) / 32) * 32;
-        int64_t grid = n_seams;
-        const int64_t cap = (int64_t)sm_count() * 32;
-        if (grid > cap) grid = cap;
-        seam_direct_kernel<<<(int)grid, threads, 0, st>>>(src, n_seams, t.T, t.B, t.overlap, (float)inv_b, out);
+        const int sms = sm_count();
+        if (n_seams >= 4LL * sms) {
+            // many seams: a warp each
+            int64_t grid = (n_seams * 32 + 255) / 256;
+            if (grid > (int64_t)sms * 16) grid = (int64_t)sms * 16;
+            seam_direct_warp_kernel<<<(int)grid, 256, 0, st>>>(src, n_seams, t.T, t.B, t.overlap, (float)inv_b,
+                                                                out);
+        } else {
+            // few seams: a CTA each, a thread per overlap entry
+            const int oo = t.overlap * t.overlap;
+            const int threads = oo >= 256 ? 256 : ((oo + 31) / 32) * 32;
+            seam_direct_kernel<<<(int)n_seams, threads, 0, st>>>(src, n_seams, t.T, t.B, t.overlap, (float)inv_b,
+                                                                 out);
+        }
     } else {
         if (n_seams > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
         seam_finalize_kernel<<<(unsigned)n_seams, 256, 0, st>>>(src, t.overlap * t.overlap, chunks,
