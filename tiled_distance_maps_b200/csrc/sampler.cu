@@ -430,13 +430,13 @@ cudaError_t launch_ddim_step(const StepCoef *coef, int step, float *maps, const 
 }
 
 template <bool U, bool E, bool I>
-static cudaError_t run_variant(const RunArgs &a, int grid, size_t smem, cudaStream_t st) {
+static cudaError_t run_variant(const RunArgs &a, int grid, int threads, size_t smem, cudaStream_t st) {
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(ddim_run_kernel<U, E, I>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    ddim_run_kernel<U, E, I><<<grid, 256, smem, st>>>(a);
+    ddim_run_kernel<U, E, I><<<grid, threads, smem, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -462,21 +462,28 @@ cudaError_t launch_ddim_run(const StepCoef *coef, int S, int first, int n_steps,
     a.cc = (1.0f + w) * s_c;
     a.cu = w * s_u;
     a.K = philox_keys(seed);
-    const int64_t grid64 = (a.total_warps + 7) / 8;
+    // a launch too small to give every SM several 8-warp CTAs runs 2-warp CTAs
+    // instead, spreading its warps over more SMs (fewer warps per scheduler:
+    // the run is then latency-bound, not issue-bound)
+    int sms = 148, dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int wpc = a.total_warps >= 4LL * 8 * sms ? 8 : 2;
+    const int64_t grid64 = (a.total_warps + wpc - 1) / wpc;
     if (grid64 > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
     const int grid = (int)grid64;
     const size_t smem = (size_t)S * (2 * sizeof(float4) + (has_eta ? sizeof(float2) : 0));
     const bool has_u = w != 0.0f;
     if (has_u) {
-        if (has_eta) return init_noise ? run_variant<true, true, true>(a, grid, smem, st)
-                                       : run_variant<true, true, false>(a, grid, smem, st);
-        return init_noise ? run_variant<true, false, true>(a, grid, smem, st)
-                          : run_variant<true, false, false>(a, grid, smem, st);
+        if (has_eta) return init_noise ? run_variant<true, true, true>(a, grid, 32 * wpc, smem, st)
+                                       : run_variant<true, true, false>(a, grid, 32 * wpc, smem, st);
+        return init_noise ? run_variant<true, false, true>(a, grid, 32 * wpc, smem, st)
+                          : run_variant<true, false, false>(a, grid, 32 * wpc, smem, st);
     }
-    if (has_eta) return init_noise ? run_variant<false, true, true>(a, grid, smem, st)
-                                   : run_variant<false, true, false>(a, grid, smem, st);
-    return init_noise ? run_variant<false, false, true>(a, grid, smem, st)
-                      : run_variant<false, false, false>(a, grid, smem, st);
+    if (has_eta) return init_noise ? run_variant<false, true, true>(a, grid, 32 * wpc, smem, st)
+                                   : run_variant<false, true, false>(a, grid, 32 * wpc, smem, st);
+    return init_noise ? run_variant<false, false, true>(a, grid, 32 * wpc, smem, st)
+                      : run_variant<false, false, false>(a, grid, 32 * wpc, smem, st);
 }
 
 }  // namespace tdm
