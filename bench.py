@@ -72,7 +72,8 @@ def alu_peak_ops(sms: int = 148, clock_ghz: float = 1.965) -> float:
 
 # the files that hold each kernel's device code (a change to them voids the
 # DRAM traffic recorded by an earlier ncu capture)
-RUN_SOURCES = ["tiled_distance_maps_b200/csrc/sampler.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
+RUN_SOURCES = ["tiled_distance_maps_b200/csrc/sampler.cu", "tiled_distance_maps_b200/csrc/noise.cuh",
+               "tiled_distance_maps_b200/csrc/common.cuh"]
 REFINE_SOURCES = ["tiled_distance_maps_b200/csrc/refine.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
 DRIFT_SOURCES = ["tiled_distance_maps_b200/csrc/drift.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
 STITCH_SOURCES = ["tiled_distance_maps_b200/csrc/stitch.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
@@ -107,20 +108,29 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled around the timed region.
+
+    The sampler starts before the warm-up and waits for its first line, since
+    nvidia-smi takes a while to start.  Each line is stamped on arrival; the
+    summary takes the lines stamped inside the timed region, plus the nearest
+    one on either side (at most one sampling interval away), so that a region
+    shorter than the interval still has its clocks."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, interval_ms: int = 50):
         self.dev = device_index
+        self.interval = interval_ms / 1000.0
+        self.ms = interval_ms
         self.proc = None
-        self.lines = []
+        self.lines = []            # (arrival time, line)
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.ms)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.th = threading.Thread(target=self._read, daemon=True)
             self.th.start()
@@ -130,7 +140,22 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def _wait(self, cond, timeout):
+        end = time.monotonic() + timeout
+        while self.proc is not None and not cond() and time.monotonic() < end and self.proc.poll() is None:
+            time.sleep(0.005)
+
+    def wait_first(self, timeout: float = 5.0):
+        self._wait(lambda: len(self.lines) > 0, timeout)
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_stop(self):
+        self.t1 = time.monotonic()
+        self._wait(lambda: len(self.lines) > 0 and self.lines[-1][0] > self.t1, 1.0 + 4 * self.interval)
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -140,10 +165,18 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
+    def _window(self):
+        if self.t0 is None or self.t1 is None:
+            return [ln for _, ln in self.lines]
+        inside = [ln for t, ln in self.lines if self.t0 <= t <= self.t1]
+        before = [ln for t, ln in self.lines if self.t0 - self.interval <= t < self.t0][-1:]
+        after = [ln for t, ln in self.lines if self.t1 < t <= self.t1 + self.interval][:1]
+        return before + inside + after
+
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in self._window():
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -272,20 +305,22 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    flags = tdm.ctx_sync(ctx)
-
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clocks:
+        clocks.wait_first()
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        flags = tdm.ctx_sync(ctx)
         barrier()
         torch.cuda.synchronize()
+        clocks.mark_start()
         start.record(stream)
         for i in range(args.steps):
             step(i)
         stop.record(stream)
         torch.cuda.synchronize()
+        clocks.mark_stop()
         barrier()
     ms = start.elapsed_time(stop)
     run_ms = [ev_run[2 * i].elapsed_time(ev_run[2 * i + 1]) for i in range(args.steps)]
@@ -433,7 +468,7 @@ def run_ours(args, rank, world, local_rank):
                          "peak_kind": "derived: 148 SMs x 128 lanes x max SM clock",
                          "ms_per_launch": run_avg_ms,
                          "ops_per_launch": ops},
-            "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"]},
+            "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"], "samples": clk["samples"]},
             "e2e": {"value": map_steps * args.steps / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": x0_host.numel() * 4,
                     "d2h_bytes_per_step": (n_maps * 195 + (T - 1)) * 4,

@@ -1,6 +1,8 @@
-"""Helpers for the GPU parity tests (tolerances, device transfers)."""
+"""Helpers for the GPU parity tests (tolerances, device transfers, inputs)."""
 import numpy as np
 import pytest
+
+import synth
 
 torch = pytest.importorskip("torch")
 
@@ -37,3 +39,12 @@ def assert_maps_close(g, o, tol=TOL_MAP, what="maps"):
     worst = np.unravel_index(np.argmax(e), e.shape)
     assert e.max() <= tol, f"{what}: normwise error {e.max():.3e} > {tol:.1e} at {worst}"
     return e.max()
+
+
+def x0_disagreeing(seed, C, T):
+    """Chain reference maps plus a symmetric per-tile perturbation, so that the
+    overlap blocks of adjacent tiles differ and the projection's x0 term is
+    exercised (the chain maps alone agree on every overlap)."""
+    x0 = synth.chain_x0(seed, C, T).astype(np.float64)
+    p = np.random.default_rng([seed, 404]).uniform(-0.5, 0.5, size=x0.shape)
+    return (x0 + 0.5 * (p + np.swapaxes(p, -1, -2))).astype(np.float32)

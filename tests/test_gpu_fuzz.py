@@ -1,7 +1,9 @@
 """Seeded random configurations of the fused run against the float64 oracle:
 chains, tiles, samples, overlap (multiple of 4), projection interval, step
 count, eta, guidance weight and the noise scales, with sample shards (b_offset,
-B_total) and noise-id offsets, at sizes the oracle finishes in a second."""
+B_total) and noise-id offsets, at sizes the oracle finishes in a second.  Half
+the configurations perturb x0 so that tile overlaps disagree; each compares the
+final maps and one state before the last step."""
 import numpy as np
 import pytest
 
@@ -42,6 +44,9 @@ def test_random_fused_runs(tdm, k):
     t = tdm.Tiling(C=C, T=T, B=B, overlap=o, sync_every=c["K"], B_total=B_total, b_offset=c["boff"],
                    sample_id_base=c["base"])
     x0 = synth.chain_x0(k, C, T, overlap=o) * float(1 + k % 3)
+    if k % 2:   # overlaps that disagree between tiles
+        p = np.random.default_rng([k, 505]).uniform(-0.5, 0.5, size=x0.shape)
+        x0 = (x0 + 0.5 * (p + np.swapaxes(p, -1, -2))).astype(np.float32)
     sch = tdm.Schedule(c["S"], eta=c["eta"])
     b_index = np.arange(c["boff"], c["boff"] + B)
     if c["init"]:
@@ -50,11 +55,19 @@ def test_random_fused_runs(tdm, k):
     else:
         x_T = synth.gaussian_maps(k + 100, C * T * B).reshape(C, T, B, 64, 64) * 2.0
         maps = dev(x_T).reshape(-1).clone()
+    start = maps.clone()
     tdm.ddim_run(sch, maps, dev(x0), c["w"], c["s_c"], c["s_u"], c["seed"], t, init_noise=c["init"])
-    ref = o_run(x0, osched.Schedule(S=c["S"], eta=c["eta"]), c["w"], c["s_c"], c["s_u"], c["seed"], b_index,
-                B_total, overlap=o, sync_every=c["K"], sample_id_base=c["base"], x_T=x_T)
+    ref, traj = o_run(x0, osched.Schedule(S=c["S"], eta=c["eta"]), c["w"], c["s_c"], c["s_u"], c["seed"], b_index,
+                      B_total, overlap=o, sync_every=c["K"], sample_id_base=c["base"], x_T=x_T,
+                      return_trajectory=True)
     got = host(maps).reshape(C, T, B, 64, 64)
     assert_maps_close(got, ref, TOL_MAP, f"config {c}")
+    if c["S"] > 1:
+        # a state before the last step (the last step alone sets the final maps)
+        m = 1 + k % (c["S"] - 1)
+        tdm.ddim_run(sch, start, dev(x0), c["w"], c["s_c"], c["s_u"], c["seed"], t, init_noise=c["init"],
+                     first_step=c["S"] - 1, n_steps=m)
+        assert_maps_close(host(start).reshape(C, T, B, 64, 64), traj[m - 1], TOL_MAP, f"config {c}, {m} steps")
 
 
 @pytest.mark.parametrize("k", range(24))

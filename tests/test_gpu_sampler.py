@@ -7,7 +7,8 @@ import synth
 from oracle import philox, schedule as osched
 from oracle.ddim import (ddim_run as o_run, eps_standin as o_eps, init_noise as o_init,
                          sample_ids, stream_noise)
-from tests.gpu_util import (TOL_MAP, Z_ABS_ERR, assert_maps_close, dev, host, needs_gpu, normwise, torch)
+from tests.gpu_util import (TOL_MAP, Z_ABS_ERR, assert_maps_close, dev, host, needs_gpu, normwise, torch,
+                            x0_disagreeing)
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
@@ -284,11 +285,40 @@ def test_ddpm_ancestral_sampler_1000_steps(tdm):
     assert_maps_close(_as5(maps, t), x, TOL_MAP, "DDPM run")
 
 
+@pytest.mark.parametrize("S,K,eta,w", [(10, 1, 0.0, 1.0), (10, 3, 1.0, 0.0), (20, 2, 1.0, 1.0), (8, 0, 0.0, 1.0)])
+def test_fused_run_intermediate_states(tdm, S, K, eta, w):
+    # The stand-in's last step (alpha_bar_prev = 1) gives x0 plus that step's
+    # own noise whatever the state before it, so final maps alone do not see
+    # the trajectory: the states after m < S steps are compared here, from a
+    # single run of m steps and from runs resumed in parts.
+    C, T, B = 2, 3, 4
+    t = tdm.Tiling(C=C, T=T, B=B, overlap=12, sync_every=K)
+    sch = tdm.Schedule(S, eta=eta)
+    x0 = x0_disagreeing(11, C, T)
+    x0d = dev(x0).reshape(-1)
+    _, traj = o_run(x0, osched.Schedule(S=S, eta=eta), w, 0.1, 0.3, 9, np.arange(B), B, overlap=12, sync_every=K,
+                    return_trajectory=True)
+    for m in (1, 2, S // 2, S - 1, S):
+        maps = _maps(t)
+        tdm.ddim_run(sch, maps, x0d, w, 0.1, 0.3, 9, t, first_step=S - 1, n_steps=m)
+        assert_maps_close(_as5(maps, t), traj[m - 1], TOL_MAP, f"state after {m} of {S} steps")
+    for cuts in ((1,), (S // 3, S // 2)):
+        parts, done = _maps(t), 0
+        for n in list(cuts) + [S - 1]:
+            tdm.ddim_run(sch, parts, x0d, w, 0.1, 0.3, 9, t, init_noise=done == 0, first_step=S - 1 - done,
+                         n_steps=n - done)
+            done = n
+        assert_maps_close(_as5(parts, t), traj[S - 2], TOL_MAP, f"state after {S - 1} steps, cut at {cuts}")
+
+
 @pytest.mark.parametrize("S,K,eta,w,cuts", [(10, 1, 0.0, 1.0, (4,)), (10, 3, 1.0, 0.0, (2, 7)),
                                             (8, 0, 0.0, 1.0, (5,)), (20, 3, 1.0, 1.0, (1, 10, 19))])
 def test_fused_run_resumes_bit_exactly(tdm, S, K, eta, w, cuts):
     # the run split after the given numbers of steps, the state kept in the
-    # maps between the parts, equals the whole run bit for bit
+    # maps between the parts, ends on the whole run's final maps bit for bit
+    # (the last step sets them from x0, its own noise and, where projected,
+    # the partner's; test_fused_run_intermediate_states covers the states
+    # before it)
     t = tdm.Tiling(C=2, T=3, B=4, overlap=12, sync_every=K)
     sch = tdm.Schedule(S, eta=eta)
     x0 = dev(synth.chain_x0(2, 2, 3)).reshape(-1)

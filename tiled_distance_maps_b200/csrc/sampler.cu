@@ -5,7 +5,7 @@
 // reduced step count (§4.1, §5.1.1) with classifier-free guidance (§3.1, ref.
 // [15]); tiled regions are coupled only through the overlap projection of
 // §4.3.2.  The stand-in eps is the ideal denoiser toward x0 plus Philox noise.
-#include "common.cuh"
+#include "noise.cuh"
 
 namespace tdm {
 namespace {
@@ -193,51 +193,49 @@ __device__ __forceinline__ LaneCounter lane_counter(int r, int q, uint64_t g, co
     return L;
 }
 
-// The normals of NS streams (tags TAGS...) of one step for one lane: the
-// streams share counter words 0 and 1, so round 2's first product is shared.
-template <int NS>
-__device__ __forceinline__ void lane_normals(const LaneCounter &L, uint32_t step_word, const int (&tags)[NS],
-                                             const PhiloxKeys &K, float4 (&z)[NS]) {
-    const uint64_t p0 = (uint64_t)Philox::M0 * (L.A ^ step_word);
-    const uint32_t w2 = (uint32_t)(p0 >> 32) ^ L.L0 ^ K.k1[1];
-    const uint32_t w3 = (uint32_t)p0;
-#pragma unroll
-    for (int s = 0; s < NS; ++s) {
-        const uint64_t p1 = (uint64_t)Philox::M1 * (L.B ^ ((uint32_t)tags[s] << 24));
-        uint4 c = make_uint4((uint32_t)(p1 >> 32) ^ L.L1 ^ K.k0[1], (uint32_t)p1, w2, w3);
-        c = philox_rounds<2>(c, K);
-        z[s] = words_to_normals(c);
-    }
+// Round-2 output words 0 and 1 of stream tag t: the product of round-1 word 2
+// (B ^ t << 24) carries the tag but not the step word, so it is computed once
+// per lane and stream.
+__device__ __forceinline__ uint2 round2_xy(const LaneCounter &L, int tag, const PhiloxKeys &K) {
+    const uint64_t p1 = (uint64_t)Philox::M1 * (L.B ^ ((uint32_t)tag << 24));
+    return make_uint2((uint32_t)(p1 >> 32) ^ L.L1 ^ K.k0[1], (uint32_t)p1);
 }
 
-// The same draws as lane_normals, as negated packed halves (box_muller_packed).
+// The draws of NS streams of one step for one lane (xy: round2_xy of each
+// stream), as the radius and angle parts of box_muller_packed, each stream's
+// term nk[s] rho (cos | sin) added to (a02, a13) as soon as it is drawn.
+// Round 2's product of word 0 (A ^ step word) is shared by the streams.
 template <int NS>
-__device__ __forceinline__ void lane_normals_packed(const LaneCounter &L, uint32_t step_word, const int (&tags)[NS],
-                                                    const PhiloxKeys &K, float2 (&zc)[NS], float2 (&zs)[NS]) {
+__device__ __forceinline__ void lane_noise_packed(const LaneCounter &L, uint32_t step_word, const uint2 (&xy)[NS],
+                                                  const PhiloxKeys &K, const float2 (&nk)[NS], float2 &a02,
+                                                  float2 &a13) {
     const uint64_t p0 = (uint64_t)Philox::M0 * (L.A ^ step_word);
     const uint32_t w2 = (uint32_t)(p0 >> 32) ^ L.L0 ^ K.k1[1];
     const uint32_t w3 = (uint32_t)p0;
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
-        const uint64_t p1 = (uint64_t)Philox::M1 * (L.B ^ ((uint32_t)tags[s] << 24));
-        uint4 c = make_uint4((uint32_t)(p1 >> 32) ^ L.L1 ^ K.k0[1], (uint32_t)p1, w2, w3);
-        c = philox_rounds<2>(c, K);
-        box_muller_packed(c, zc[s], zs[s]);
+        const uint4 c = philox_rounds<2>(make_uint4(xy[s].x, xy[s].y, w2, w3), K);
+        float2 rho, cs, sn;
+        box_muller_packed(c, rho, cs, sn);
+        const float2 t = __fmul2_rn(nk[s], rho);
+        a02 = __ffma2_rn(t, cs, a02);
+        a13 = __ffma2_rn(t, sn, a13);
     }
 }
 
 template <bool HAS_U, bool HAS_ETA, bool INIT>
 __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
-    // per step, packed (both halves equal): (ka, kx0) then (-kc, -ku), the noise
-    // coefficients negated for the negated packed normals; then [S] -ks
+    // per step, packed (both halves equal): (ka, kx0) then (-kc, -ku) kRadScale,
+    // the noise coefficients times the factor z = -kRadScale rho cos (sin) of
+    // box_muller_packed's parts; then [S] -ks kRadScale
     extern __shared__ float4 sco[];
     float2 *sks = reinterpret_cast<float2 *>(sco + 2 * a.S);
     for (int i = threadIdx.x; i < a.S; i += blockDim.x) {
         const StepCoef c = a.coef[i];
-        const float kc = c.kb * a.cc, ku = -(c.kb * a.cu);
+        const float nkc = -(c.kb * a.cc) * kRadScale, nku = (c.kb * a.cu) * kRadScale;
         sco[2 * i] = make_float4(c.ka, c.ka, c.kx0, c.kx0);
-        sco[2 * i + 1] = make_float4(-kc, -kc, -ku, -ku);
-        if (HAS_ETA) sks[i] = make_float2(-c.ks, -c.ks);
+        sco[2 * i + 1] = make_float4(nkc, nkc, nku, nku);
+        if (HAS_ETA) sks[i] = make_float2(-c.ks * kRadScale, -c.ks * kRadScale);
     }
     __syncthreads();
 
@@ -260,11 +258,10 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     // the state as packed column pairs (x0, x2) and (x1, x3) of the quad
     float2 x02, x13;
     if (INIT) {
-        constexpr int kInit[1] = {TDM_STREAM_INIT};
-        float2 zc[1], zs[1];
-        lane_normals_packed<1>(L, 0u, kInit, a.K, zc, zs);
-        x02 = __fmul2_rn(zc[0], make_float2(-1.0f, -1.0f));
-        x13 = __fmul2_rn(zs[0], make_float2(-1.0f, -1.0f));
+        const uint2 xy[1] = {round2_xy(L, TDM_STREAM_INIT, a.K)};
+        const float2 nk[1] = {make_float2(-kRadScale, -kRadScale)};
+        x02 = x13 = make_float2(0.0f, 0.0f);
+        lane_noise_packed<1>(L, 0u, xy, a.K, nk, x02, x13);
     } else {
         const float4 x = ld4(mp + r * kN + 4 * q);
         x02 = make_float2(x.x, x.z);
@@ -275,32 +272,32 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     // the projection follows the steps counted from the start of the whole
     // run, so a run resumed at step `first` projects where the whole run would
     int until_sync = a.sync_every > 0 ? a.sync_every - (a.S - 1 - a.first) % a.sync_every : 0;
+    // the state is stepped as y = x - gam x0 (the loop's x02, x13), so the x0
+    // term of every step is one scalar update of gam: x' = ka x + kx0 x0 + n
+    // gives y' = ka y + n and gam' = ka gam + kx0; x = y + gam x0 at the end.
+    // The projection averages x over a pair: y' = (y + y_o) / 2 + gam d with
+    // d = (x0_o - x0) / 2 (zero where the two tiles' x0 agree).
+    float gam = 0.0f;
 
     constexpr int NS = 1 + (HAS_U ? 1 : 0) + (HAS_ETA ? 1 : 0);
     constexpr int kTags[3] = {TDM_STREAM_EPS_C, HAS_U ? TDM_STREAM_EPS_U : TDM_STREAM_ETA, TDM_STREAM_ETA};
-    int tags[NS];
+    uint2 xy[NS];
 #pragma unroll
-    for (int s = 0; s < NS; ++s) tags[s] = kTags[s];
+    for (int s = 0; s < NS; ++s) xy[s] = round2_xy(L, kTags[s], a.K);
 
     for (int i = a.first; i >= a.last; --i) {
         const float4 c0 = sco[2 * i], c1 = sco[2 * i + 1];
-        const float2 ka = make_float2(c0.x, c0.y), kx0 = make_float2(c0.z, c0.w);
+        const float2 ka = make_float2(c0.x, c0.y);
         const float2 nkc = make_float2(c1.x, c1.y), nku = make_float2(c1.z, c1.w);
-        float2 zc[NS], zs[NS];
-        lane_normals_packed<NS>(L, (uint32_t)i, tags, a.K, zc, zs);
-        float2 a02 = __ffma2_rn(nkc, zc[0], __fmul2_rn(kx0, r02));
-        float2 a13 = __ffma2_rn(nkc, zs[0], __fmul2_rn(kx0, r13));
-        if (HAS_U) {
-            a02 = __ffma2_rn(nku, zc[1], a02);
-            a13 = __ffma2_rn(nku, zs[1], a13);
-        }
-        if (HAS_ETA) {
-            const float2 nks = sks[i];
-            a02 = __ffma2_rn(nks, zc[NS - 1], a02);
-            a13 = __ffma2_rn(nks, zs[NS - 1], a13);
-        }
+        float2 nk[NS];
+        nk[0] = nkc;
+        if (HAS_U) nk[1] = nku;
+        if (HAS_ETA) nk[NS - 1] = sks[i];
+        float2 a02 = make_float2(0.f, 0.f), a13 = make_float2(0.f, 0.f);
+        lane_noise_packed<NS>(L, (uint32_t)i, xy, a.K, nk, a02, a13);
         x02 = __ffma2_rn(ka, x02, a02);
         x13 = __ffma2_rn(ka, x13, a13);
+        gam = fmaf(c0.x, gam, c0.z);
         if (sync_warp && --until_sync == 0) {
             until_sync = a.sync_every;
             float2 o02, o13;
@@ -308,12 +305,22 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
             o02.y = __shfl_xor_sync(0xffffffffu, x02.y, 16);
             o13.x = __shfl_xor_sync(0xffffffffu, x13.x, 16);
             o13.y = __shfl_xor_sync(0xffffffffu, x13.y, 16);
+            float2 d02, d13;
+            d02.x = __shfl_xor_sync(0xffffffffu, r02.x, 16);
+            d02.y = __shfl_xor_sync(0xffffffffu, r02.y, 16);
+            d13.x = __shfl_xor_sync(0xffffffffu, r13.x, 16);
+            d13.y = __shfl_xor_sync(0xffffffffu, r13.y, 16);
             if (paired) {
-                x02 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x02, o02));
-                x13 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x13, o13));
+                d02 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(d02, make_float2(-r02.x, -r02.y)));
+                d13 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(d13, make_float2(-r13.x, -r13.y)));
+                const float2 g2 = make_float2(gam, gam);
+                x02 = __ffma2_rn(g2, d02, __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x02, o02)));
+                x13 = __ffma2_rn(g2, d13, __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x13, o13)));
             }
         }
     }
+    x02 = __ffma2_rn(make_float2(gam, gam), r02, x02);
+    x13 = __ffma2_rn(make_float2(gam, gam), r13, x13);
     const float4 x = make_float4(x02.x, x13.x, x02.y, x13.y);
 
     // unfold: the quad's upper entries go to (r, j) and their mirrors to (j, r)
