@@ -341,3 +341,31 @@ def test_fused_run_step_range_is_checked(tdm):
     for first, n, init in ((10, 1, False), (-1, 1, False), (5, 7, False), (5, 0, False), (5, 2, True)):
         with pytest.raises(tdm.TdmError):
             tdm.ddim_run(sch, m, x0, 0.0, 0.1, 0.0, 0, t, init_noise=init, first_step=first, n_steps=n)
+
+
+def test_large_and_small_launch_shapes_agree(tdm):
+    # A launch of at least 4 x 8 warps per SM runs 8-warp CTAs with the
+    # warp-voted series; a smaller one runs 2-warp CTAs with the series
+    # selected per pair.  Both give the same bits, and the large one matches
+    # the oracle (final maps and a state before the last step).
+    import torch as _t
+    sms = _t.cuda.get_device_properties(0).multi_processor_count
+    T, S = 4, 10
+    B = -(-4 * 8 * sms // (17 * T))          # enough chain-samples for 8-warp CTAs
+    t_big = tdm.Tiling(C=1, T=T, B=B, overlap=12, sync_every=1)
+    sch = tdm.Schedule(S)
+    x0 = x0_disagreeing(21, 1, T)
+    x0d = dev(x0).reshape(-1)
+    big = _maps(t_big)
+    tdm.ddim_run(sch, big, x0d, 1.0, 0.1, 0.3, 4, t_big)
+    part = _maps(t_big)
+    tdm.ddim_run(sch, part, x0d, 1.0, 0.1, 0.3, 4, t_big, first_step=S - 1, n_steps=S - 1)
+    for off in (0, B - 3):
+        t_small = tdm.Tiling(C=1, T=T, B=3, overlap=12, sync_every=1, B_total=B, b_offset=off)
+        small = _maps(t_small)
+        tdm.ddim_run(sch, small, x0d, 1.0, 0.1, 0.3, 4, t_small)
+        np.testing.assert_array_equal(_as5(small, t_small), _as5(big, t_big)[:, :, off:off + 3])
+    ref, traj = o_run(x0, osched.Schedule(S=S), 1.0, 0.1, 0.3, 4, np.arange(B), B, overlap=12, sync_every=1,
+                      return_trajectory=True)
+    assert_maps_close(_as5(big, t_big), ref, TOL_MAP, "large launch, final maps")
+    assert_maps_close(_as5(part, t_big), traj[S - 2], TOL_MAP, "large launch, state before the last step")

@@ -128,16 +128,19 @@ __device__ __forceinline__ float2 box_muller(uint32_t a, uint32_t b) {
 // instruction, each rounded as the scalar operation, so rho, cs and sn are
 // bit-identical to box_muller_parts'):  z0 = -kRadScale rho.x cs.x,
 // z1 = -kRadScale rho.x sn.x, z2 = -kRadScale rho.y cs.y,
-// z3 = -kRadScale rho.y sn.y.  The series branch runs only when a lane of the
-// warp needs it (about one call in nine at e < 2^-9), decided by a warp vote:
-// all 32 lanes must call together.
+// z3 = -kRadScale rho.y sn.y.  With VOTE the series branch runs only when a
+// lane of the warp needs it (about one call in nine at e < 2^-9), decided by
+// a warp vote, and all 32 lanes must call together; without it the series is
+// computed for every pair and selected, which keeps the branch off each
+// lane's dependency chain (for launches too small to hide latency).
+template <bool VOTE>
 __device__ __forceinline__ void box_muller_packed(uint4 w, float2 &rho, float2 &cs, float2 &sn) {
     const float2 f = make_float2(mantissa_float(w.x), mantissa_float(w.z));
     const float2 fb = make_float2(mantissa_float(w.y), mantissa_float(w.w));
     const float2 u1 = __ffma2_rn(f, make_float2(-1.0f, -1.0f), make_float2(2.0f, 2.0f));     // 2 - f, exact
     float2 v = make_float2(-mufu_lg2(u1.x), -mufu_lg2(u1.y));
     const bool sx = f.x < kSerEdge, sy = f.y < kSerEdge;
-    if (__any_sync(0xffffffffu, sx || sy)) {
+    if (!VOTE || __any_sync(0xffffffffu, sx || sy)) {
         const float2 e = __fadd2_rn(f, make_float2(-1.0f, -1.0f));
         const float2 ser = __fmul2_rn(
             e, __ffma2_rn(e, __ffma2_rn(e, make_float2(0x1.ec709ep-2f, 0x1.ec709ep-2f),

@@ -205,7 +205,7 @@ __device__ __forceinline__ uint2 round2_xy(const LaneCounter &L, int tag, const 
 // stream), as the radius and angle parts of box_muller_packed, each stream's
 // term nk[s] rho (cos | sin) added to (a02, a13) as soon as it is drawn.
 // Round 2's product of word 0 (A ^ step word) is shared by the streams.
-template <int NS>
+template <int NS, bool VOTE>
 __device__ __forceinline__ void lane_noise_packed(const LaneCounter &L, uint32_t step_word, const uint2 (&xy)[NS],
                                                   const PhiloxKeys &K, const float2 (&nk)[NS], float2 &a02,
                                                   float2 &a13) {
@@ -216,14 +216,18 @@ __device__ __forceinline__ void lane_noise_packed(const LaneCounter &L, uint32_t
     for (int s = 0; s < NS; ++s) {
         const uint4 c = philox_rounds<2>(make_uint4(xy[s].x, xy[s].y, w2, w3), K);
         float2 rho, cs, sn;
-        box_muller_packed(c, rho, cs, sn);
+        box_muller_packed<VOTE>(c, rho, cs, sn);
         const float2 t = __fmul2_rn(nk[s], rho);
         a02 = __ffma2_rn(t, cs, a02);
         a13 = __ffma2_rn(t, sn, a13);
     }
 }
 
-template <bool HAS_U, bool HAS_ETA, bool INIT>
+// WIDE: 8-warp CTAs of a launch large enough to be throughput-bound (the
+// series behind a warp vote, the partner's x0 exchanged at each projection
+// to save registers); otherwise 2-warp CTAs of a latency-bound launch (the
+// series selected per pair, the x0 term of the projection formed once).
+template <bool HAS_U, bool HAS_ETA, bool INIT, bool WIDE>
 __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     // per step, packed (both halves equal): (ka, kx0) then (-kc, -ku) kRadScale,
     // the noise coefficients times the factor z = -kRadScale rho cos (sin) of
@@ -261,7 +265,7 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
         const uint2 xy[1] = {round2_xy(L, TDM_STREAM_INIT, a.K)};
         const float2 nk[1] = {make_float2(-kRadScale, -kRadScale)};
         x02 = x13 = make_float2(0.0f, 0.0f);
-        lane_noise_packed<1>(L, 0u, xy, a.K, nk, x02, x13);
+        lane_noise_packed<1, WIDE>(L, 0u, xy, a.K, nk, x02, x13);
     } else {
         const float4 x = ld4(mp + r * kN + 4 * q);
         x02 = make_float2(x.x, x.z);
@@ -278,6 +282,16 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     // The projection averages x over a pair: y' = (y + y_o) / 2 + gam d with
     // d = (x0_o - x0) / 2 (zero where the two tiles' x0 agree).
     float gam = 0.0f;
+    float2 d02 = make_float2(0.f, 0.f), d13 = make_float2(0.f, 0.f);
+    const auto half_x0_gap = [&]() {    // (x0 of the partner - x0) / 2
+        d02.x = __shfl_xor_sync(0xffffffffu, r02.x, 16);
+        d02.y = __shfl_xor_sync(0xffffffffu, r02.y, 16);
+        d13.x = __shfl_xor_sync(0xffffffffu, r13.x, 16);
+        d13.y = __shfl_xor_sync(0xffffffffu, r13.y, 16);
+        d02 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(d02, make_float2(-r02.x, -r02.y)));
+        d13 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(d13, make_float2(-r13.x, -r13.y)));
+    };
+    if (!WIDE && sync_warp) half_x0_gap();
 
     constexpr int NS = 1 + (HAS_U ? 1 : 0) + (HAS_ETA ? 1 : 0);
     constexpr int kTags[3] = {TDM_STREAM_EPS_C, HAS_U ? TDM_STREAM_EPS_U : TDM_STREAM_ETA, TDM_STREAM_ETA};
@@ -294,7 +308,7 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
         if (HAS_U) nk[1] = nku;
         if (HAS_ETA) nk[NS - 1] = sks[i];
         float2 a02 = make_float2(0.f, 0.f), a13 = make_float2(0.f, 0.f);
-        lane_noise_packed<NS>(L, (uint32_t)i, xy, a.K, nk, a02, a13);
+        lane_noise_packed<NS, WIDE>(L, (uint32_t)i, xy, a.K, nk, a02, a13);
         x02 = __ffma2_rn(ka, x02, a02);
         x13 = __ffma2_rn(ka, x13, a13);
         gam = fmaf(c0.x, gam, c0.z);
@@ -305,14 +319,8 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
             o02.y = __shfl_xor_sync(0xffffffffu, x02.y, 16);
             o13.x = __shfl_xor_sync(0xffffffffu, x13.x, 16);
             o13.y = __shfl_xor_sync(0xffffffffu, x13.y, 16);
-            float2 d02, d13;
-            d02.x = __shfl_xor_sync(0xffffffffu, r02.x, 16);
-            d02.y = __shfl_xor_sync(0xffffffffu, r02.y, 16);
-            d13.x = __shfl_xor_sync(0xffffffffu, r13.x, 16);
-            d13.y = __shfl_xor_sync(0xffffffffu, r13.y, 16);
+            if (WIDE) half_x0_gap();
             if (paired) {
-                d02 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(d02, make_float2(-r02.x, -r02.y)));
-                d13 = __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(d13, make_float2(-r13.x, -r13.y)));
                 const float2 g2 = make_float2(gam, gam);
                 x02 = __ffma2_rn(g2, d02, __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x02, o02)));
                 x13 = __ffma2_rn(g2, d13, __fmul2_rn(make_float2(0.5f, 0.5f), __fadd2_rn(x13, o13)));
@@ -436,15 +444,22 @@ cudaError_t launch_ddim_step(const StepCoef *coef, int step, float *maps, const 
     return cudaGetLastError();
 }
 
-template <bool U, bool E, bool I>
-static cudaError_t run_variant(const RunArgs &a, int grid, int threads, size_t smem, cudaStream_t st) {
+template <bool U, bool E, bool I, bool V>
+static cudaError_t run_variant4(const RunArgs &a, int grid, int threads, size_t smem, cudaStream_t st) {
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(ddim_run_kernel<U, E, I>,
+        cudaError_t e = cudaFuncSetAttribute(ddim_run_kernel<U, E, I, V>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    ddim_run_kernel<U, E, I><<<grid, threads, smem, st>>>(a);
+    ddim_run_kernel<U, E, I, V><<<grid, threads, smem, st>>>(a);
     return cudaGetLastError();
+}
+
+// 8-warp CTAs: the WIDE kernel; 2-warp CTAs (small launches): the other
+template <bool U, bool E, bool I>
+static cudaError_t run_variant(const RunArgs &a, int grid, int threads, size_t smem, cudaStream_t st) {
+    return threads == 256 ? run_variant4<U, E, I, true>(a, grid, threads, smem, st)
+                          : run_variant4<U, E, I, false>(a, grid, threads, smem, st);
 }
 
 cudaError_t launch_ddim_run(const StepCoef *coef, int S, int first, int n_steps, float *maps, const float *x0,
