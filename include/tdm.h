@@ -99,7 +99,10 @@ typedef struct tdm_tiling {
  * device), TDM_ENOMEM, TDM_ECUDA.  The calls that keep intermediate results
  * in the scratch (tdm_seam_discrepancy, tdm_nonoverlap_drift,
  * tdm_kabsch_stitch) must not overlap on the GPU for one context: issue them
- * on one stream, or give each stream its own context. */
+ * on one stream, or give each stream its own context.  Host threads may share
+ * a context (its lane-plan cache is locked), but the message of
+ * tdm_ctx_last_error is the context's last one, whichever thread failed: a
+ * thread that reads messages should have its own context. */
 tdm_status tdm_ctx_create(tdm_ctx **out, int32_t device);
 
 /* Frees everything the context owns.  NULL is ignored. */

@@ -65,10 +65,9 @@ def test_stitch_chromosome_chain_full_size(tdm):
     assert (np.abs(res[:, idx] - rref) / np.maximum(rref, 2e-5)).max() <= TOL_RESID
 
 
-def test_stitch_pairs_over_several_scratch_chunks(tdm):
-    # 4000 samples of a 32-tile chain: more (chain, sample) pairs than one
-    # chunk of tile maps in the context scratch holds; chains on both sides of
-    # a chunk boundary through the oracle
+def test_stitch_many_pairs(tdm):
+    # 4000 samples of a 32-tile chain: several waves of the one-pass kernel's
+    # CTAs; chains at the start, the middle and the end through the oracle
     C, T, B = 1, 32, 4000
     X, _, _ = synth.tile_coords(7, C, T, B, noise=0.02)
     got, res = _run(tdm, X, T, 12)
@@ -77,6 +76,27 @@ def test_stitch_pairs_over_several_scratch_chunks(tdm):
     scale = np.abs(ref).max(axis=(-1, -2))
     assert (np.abs(got[:, idx] - ref).max(axis=(-1, -2)) / scale).max() <= TOL_CHAIN
     assert (np.abs(res[:, idx] - rref) / np.maximum(rref, 2e-5)).max() <= TOL_RESID
+
+
+def test_stitch_two_pass_over_several_scratch_chunks(tdm):
+    # 520-tile chains (over the one-pass limit of 512 tiles) for 400 samples:
+    # the two-pass form, whose tile maps of 194 pairs fill one chunk of the
+    # context scratch.  Chains on both sides of each chunk boundary go through
+    # the oracle: every seam's residual, and the first 40 tiles of the chain
+    # (float32 composition over hundreds of seams drifts by about 1e-4 of the
+    # chain's extent, as test_stitch_longest_chains notes)
+    C, T, B, o = 1, 520, 400, 12
+    X, _, _ = synth.tile_coords(17, C, T, B, overlap=o, noise=0.02)
+    got, res = _run(tdm, X, T, o)
+    assert np.isfinite(got).all() and np.isfinite(res).all()
+    idx = np.array([0, 193, 194, 387, 388, 399])
+    ref, rref = ostitch.stitch(X[:, :, idx].astype(np.float64), o)
+    L40 = 64 + 39 * (64 - o)
+    scale = np.abs(ref[:, :, :L40]).max(axis=(-1, -2))
+    assert (np.abs(got[:, idx, :L40] - ref[:, :, :L40]).max(axis=(-1, -2)) / scale).max() <= TOL_CHAIN
+    assert (np.abs(res[:, idx] - rref) / np.maximum(rref, 2e-5)).max() <= TOL_RESID
+    whole = (np.abs(got[:, idx] - ref).max(axis=(-1, -2)) / np.abs(ref).max(axis=(-1, -2))).max()
+    assert whole <= 5 * TOL_CHAIN, whole
 
 
 def test_stitch_longest_chains(tdm):

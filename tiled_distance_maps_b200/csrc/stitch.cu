@@ -9,9 +9,12 @@
 // maps compose along the chain into tile 0's frame; overlap beads take the
 // mean of their two aligned copies.
 //
-// Two passes over chunks of (chain, sample) pairs whose tile maps fit the
-// context scratch: one warp per pair aligns the seams and composes the maps by
-// a shuffle scan, 32 tiles at a time; then one thread per chain bead places it.
+// Chains of up to kFusedMaxT tiles take one pass: a CTA per (chain, sample)
+// pair, whose first warp aligns the seams and composes the maps by a shuffle
+// scan, 32 tiles at a time, into shared memory, after which all its threads
+// place the pair's beads.  Longer chains take two passes over chunks of pairs
+// whose maps fit the context scratch: the same alignment into global memory,
+// then one thread per group of chain beads.
 #include "common.cuh"
 
 namespace tdm {
@@ -66,15 +69,30 @@ __device__ __forceinline__ void apply(const Rigid &g, const float *x, float *y) 
         y[i] = fmaf(g.r[3 * i], x[0], fmaf(g.r[3 * i + 1], x[1], fmaf(g.r[3 * i + 2], x[2], g.t[i])));
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float rsqrt_approx(float x) {
+    float r;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // Eigen-decomposition of a symmetric 3 x 3 matrix by cyclic Jacobi (Golub &
 // Van Loan §8.5); descending eigenvalues, eigenvectors in the columns of V.
+// The rotation's reciprocals and square roots are the hardware approximations
+// (a few ulp): the rotation stays orthogonal to float32 rounding, and the skip
+// test below keeps theta^2 finite (|theta| < 5e11).
 template <int P, int Q>
 __device__ __forceinline__ void jrot3(float (&A)[3][3], float (&V)[3][3]) {
     const float apq = A[P][Q];
     if (!(fabsf(apq) > 1e-12f * (fabsf(A[P][P]) + fabsf(A[Q][Q])))) return;
-    const float theta = (A[Q][Q] - A[P][P]) / (2.0f * apq);
-    const float t = copysignf(1.0f, theta) / (fabsf(theta) + sqrtf(fmaf(theta, theta, 1.0f)));
-    const float c = 1.0f / sqrtf(fmaf(t, t, 1.0f));
+    const float theta = (A[Q][Q] - A[P][P]) * 0.5f * rcp_approx(apq);
+    const float r2 = fmaf(theta, theta, 1.0f);
+    const float t = copysignf(rcp_approx(fabsf(theta) + r2 * rsqrt_approx(r2)), theta);
+    const float c = rsqrt_approx(fmaf(t, t, 1.0f));
     const float s = t * c;
     A[P][P] = fmaf(-t, apq, A[P][P]);
     A[Q][Q] = fmaf(t, apq, A[Q][Q]);
@@ -169,25 +187,24 @@ __device__ Rigid align_seam(const float *P, const float *Q, int o, float *rmsd) 
 #pragma unroll
         for (int a = 0; a < 3; ++a) U[a][c] = M[a][0] * V[0][c] + M[a][1] * V[1][c] + M[a][2] * V[2][c];
     // Gram-Schmidt on U's columns (largest singular value first)
-    float n0 = sqrtf(U[0][0] * U[0][0] + U[1][0] * U[1][0] + U[2][0] * U[2][0]);
-    n0 = n0 > 0.0f ? 1.0f / n0 : 0.0f;
+    float n0 = U[0][0] * U[0][0] + U[1][0] * U[1][0] + U[2][0] * U[2][0];
+    n0 = n0 > 1e-37f ? rsqrt_approx(n0) : 0.0f;
 #pragma unroll
     for (int a = 0; a < 3; ++a) U[a][0] *= n0;
     float d01 = U[0][0] * U[0][1] + U[1][0] * U[1][1] + U[2][0] * U[2][1];
 #pragma unroll
     for (int a = 0; a < 3; ++a) U[a][1] -= d01 * U[a][0];
-    float n1 = sqrtf(U[0][1] * U[0][1] + U[1][1] * U[1][1] + U[2][1] * U[2][1]);
-    n1 = n1 > 0.0f ? 1.0f / n1 : 0.0f;
+    float n1 = U[0][1] * U[0][1] + U[1][1] * U[1][1] + U[2][1] * U[2][1];
+    n1 = n1 > 1e-37f ? rsqrt_approx(n1) : 0.0f;
 #pragma unroll
     for (int a = 0; a < 3; ++a) U[a][1] *= n1;
-    const float sigma_rel = lam[0] > 0.0f ? lam[2] / lam[0] : 0.0f;
-    if (sigma_rel > 1e-10f) {
+    if (lam[0] > 0.0f && lam[2] > 1e-10f * lam[0]) {
         const float d02 = U[0][0] * U[0][2] + U[1][0] * U[1][2] + U[2][0] * U[2][2];
         const float d12 = U[0][1] * U[0][2] + U[1][1] * U[1][2] + U[2][1] * U[2][2];
 #pragma unroll
         for (int a = 0; a < 3; ++a) U[a][2] -= d02 * U[a][0] + d12 * U[a][1];
-        float n2 = sqrtf(U[0][2] * U[0][2] + U[1][2] * U[1][2] + U[2][2] * U[2][2]);
-        n2 = n2 > 0.0f ? 1.0f / n2 : 0.0f;
+        float n2 = U[0][2] * U[0][2] + U[1][2] * U[1][2] + U[2][2] * U[2][2];
+        n2 = n2 > 1e-37f ? rsqrt_approx(n2) : 0.0f;
 #pragma unroll
         for (int a = 0; a < 3; ++a) U[a][2] *= n2;
     } else {
@@ -255,19 +272,14 @@ __device__ __forceinline__ void async_copy4(float *dst, const float *src) {
                  : "memory");
 }
 
-// Pass 1: one warp (one CTA) per (chain, sample) of pairs [pair0, pair0 + n):
-// the seam beads of 32 tiles at a time staged in shared memory by coalesced
-// warp-wide asynchronous copies (per-lane stride 3o+1 floats, odd, so the lanes' reads do
-// not conflict), then every tile's map into gmaps[(pair - pair0) * T + k] and
-// the residuals into resid.
-__global__ void __launch_bounds__(32) stitch_align_kernel(const float *__restrict__ coords, int T, int B, int o,
-                                                          int64_t pair0, Rigid *__restrict__ gmaps,
-                                                          float *__restrict__ resid) {
-    extern __shared__ float sbeads[];    // [2][32][3o+1]: P then Q per lane
-    const int lane = threadIdx.x;
-    const int64_t q = blockIdx.x;
-    const int64_t pair = pair0 + q;
-    const int c = (int)(pair / B), b = (int)(pair - (int64_t)(pair / B) * B);
+// The maps of every tile of pair (c, b) into out[0 .. T) and its residuals
+// into resid (warp-wide): the seam beads of 32 tiles at a time are staged in
+// shared memory (sbeads: [2][32][3o+1], P then Q per lane) by coalesced
+// warp-wide asynchronous copies (per-lane stride 3o+1 floats, odd, so the
+// lanes' reads do not conflict); out may be global or shared memory.
+__device__ __forceinline__ void pair_maps(const float *__restrict__ coords, int T, int B, int o, int c, int b,
+                                          int64_t pair, float *sbeads, float *__restrict__ resid, Rigid *out) {
+    const int lane = threadIdx.x & 31;
     const int s = kN - o;
     const int n3 = 3 * o, ld = 3 * o + 1;
     float *sP = sbeads, *sQ = sbeads + 32 * ld;
@@ -286,8 +298,21 @@ __global__ void __launch_bounds__(32) stitch_align_kernel(const float *__restric
         asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
         __syncwarp();
         const Rigid gk = chunk_maps(sP + lane * ld, sQ + lane * ld, T, o, k0, pair, resid, carry, carry_prev);
-        if (k0 + lane < T) gmaps[q * T + k0 + lane] = gk;
+        if (k0 + lane < T) out[k0 + lane] = gk;
     }
+}
+
+// Pass 1 of the two-pass form: one warp (one CTA) per (chain, sample) of
+// pairs [pair0, pair0 + n): every tile's map into gmaps[(pair - pair0) * T + k]
+// and the residuals into resid.
+__global__ void __launch_bounds__(32) stitch_align_kernel(const float *__restrict__ coords, int T, int B, int o,
+                                                          int64_t pair0, Rigid *__restrict__ gmaps,
+                                                          float *__restrict__ resid) {
+    extern __shared__ float sbeads[];    // [2][32][3o+1]
+    const int64_t q = blockIdx.x;
+    const int64_t pair = pair0 + q;
+    const int c = (int)(pair / B), b = (int)(pair - (int64_t)(pair / B) * B);
+    pair_maps(coords, T, B, o, c, b, pair, sbeads, resid, gmaps + q * T);
 }
 
 __device__ __forceinline__ Rigid load_map(const Rigid *g) {
@@ -300,13 +325,79 @@ __device__ __forceinline__ Rigid load_map(const Rigid *g) {
     return o;
 }
 
-// Pass 2: one thread per G beads of the chains of pairs [pair0, pair0 + n).
-// Tile k owns chain positions [k s, k s + s), the last tile [k s, k s + 64);
-// the first o beads of tile k > 0 are the mean of tile k-1's and tile k's
-// aligned copies.  G = 4 needs o % 4 == 0: four beads then stay in one tile
-// and on one side of the overlap boundary, and their 12 coordinates are
-// 16-byte aligned in the tile and in the chain.  32-bit indices: a chunk holds
-// n L <= (scratch / 12T) * 64T beads, and pairs < 2^31 is checked by the caller.
+__device__ __forceinline__ Rigid smem_map(const Rigid *g) {
+    const float4 *v = reinterpret_cast<const float4 *>(g);
+    const float4 a = v[0], b = v[1], c = v[2];
+    Rigid o;
+    o.r[0] = a.x, o.r[1] = a.y, o.r[2] = a.z, o.r[3] = a.w;
+    o.r[4] = b.x, o.r[5] = b.y, o.r[6] = b.z, o.r[7] = b.w;
+    o.r[8] = c.x, o.t[0] = c.y, o.t[1] = c.z, o.t[2] = c.w;
+    return o;
+}
+
+// Chain beads [p, p + G) of pair (c, b) from its tiles' coordinates and maps
+// (maps: the pair's T maps, global when GLOBAL_MAPS, else shared).  Tile k owns
+// chain positions [k s, k s + s), the last tile [k s, k s + 64); the first o
+// beads of tile k > 0 are the mean of tile k-1's and tile k's aligned copies.
+// G = 4 needs o % 4 == 0: four beads then stay in one tile and on one side of
+// the overlap boundary, and their 12 coordinates are 16-byte aligned in the
+// tile and in the chain.
+template <int G, bool GLOBAL_MAPS>
+__device__ __forceinline__ void place_group(const float *__restrict__ coords, int T, int B, int o, int c, int b,
+                                            int p, const Rigid *maps, float *dst) {
+    const int s = kN - o;
+    int k = p / s;
+    if (k > T - 1) k = T - 1;
+    const int j = p - k * s;
+    // both rounds of loads (the tile's beads and map; for overlap beads also
+    // the previous tile's) are issued before any arithmetic
+    const bool ov = k > 0 && j < o;
+    float x[3 * G], xp[3 * G], y[3 * G];
+    const float *xk = coords + (((int64_t)c * T + k) * B + b) * (kN * 3) + 3 * j;
+    const float *xq = coords + (((int64_t)c * T + (ov ? k - 1 : k)) * B + b) * (kN * 3) + 3 * (s + j);
+    const Rigid gk = GLOBAL_MAPS ? load_map(maps + k) : smem_map(maps + k);
+    Rigid gp = gk;
+    if constexpr (G == 4) {
+#pragma unroll
+        for (int v = 0; v < 3; ++v) *reinterpret_cast<float4 *>(x + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xk) + v);
+        if (ov) {
+#pragma unroll
+            for (int v = 0; v < 3; ++v)
+                *reinterpret_cast<float4 *>(xp + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xq) + v);
+            gp = GLOBAL_MAPS ? load_map(maps + k - 1) : smem_map(maps + k - 1);
+        }
+    } else {
+#pragma unroll
+        for (int v = 0; v < 3 * G; ++v) x[v] = __ldg(xk + v);
+        if (ov) {
+#pragma unroll
+            for (int v = 0; v < 3 * G; ++v) xp[v] = __ldg(xq + v);
+            gp = GLOBAL_MAPS ? load_map(maps + k - 1) : smem_map(maps + k - 1);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < G; ++u) apply(gk, x + 3 * u, y + 3 * u);
+    if (ov) {
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+            float y1[3];
+            apply(gp, xp + 3 * u, y1);
+#pragma unroll
+            for (int d = 0; d < 3; ++d) y[3 * u + d] = 0.5f * (y1[d] + y[3 * u + d]);
+        }
+    }
+    if constexpr (G == 4) {
+#pragma unroll
+        for (int v = 0; v < 3; ++v) reinterpret_cast<float4 *>(dst)[v] = *reinterpret_cast<const float4 *>(y + 4 * v);
+    } else {
+#pragma unroll
+        for (int v = 0; v < 3 * G; ++v) dst[v] = y[v];
+    }
+}
+
+// Pass 2 of the two-pass form: one thread per G beads of the chains of pairs
+// [pair0, pair0 + n).  32-bit indices: a chunk holds n L <= (scratch / 12T) *
+// 64T beads, and pairs < 2^31 is checked by the caller.
 template <int G>
 __global__ void __launch_bounds__(256) stitch_place_kernel(const float *__restrict__ coords, int T, int B, int o,
                                                            int pair0, int n, const Rigid *__restrict__ gmaps,
@@ -320,55 +411,30 @@ __global__ void __launch_bounds__(256) stitch_place_kernel(const float *__restri
         const int p = (idx - q * LG) * G;
         const int pair = pair0 + q;
         const int c = pair / B, b = pair - (pair / B) * B;
-        int k = p / s;
-        if (k > T - 1) k = T - 1;
-        const int j = p - k * s;
-        // both rounds of loads (the tile's beads and map; for overlap beads also
-        // the previous tile's) are issued before any arithmetic
-        const bool ov = k > 0 && j < o;
-        float x[3 * G], xp[3 * G], y[3 * G];
-        const float *xk = coords + (((int64_t)c * T + k) * B + b) * (kN * 3) + 3 * j;
-        const float *xq = coords + (((int64_t)c * T + (ov ? k - 1 : k)) * B + b) * (kN * 3) + 3 * (s + j);
-        const Rigid gk = load_map(gmaps + (int64_t)q * T + k);
-        Rigid gp = gk;
-        if constexpr (G == 4) {
-#pragma unroll
-            for (int v = 0; v < 3; ++v) *reinterpret_cast<float4 *>(x + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xk) + v);
-            if (ov) {
-#pragma unroll
-                for (int v = 0; v < 3; ++v)
-                    *reinterpret_cast<float4 *>(xp + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xq) + v);
-                gp = load_map(gmaps + (int64_t)q * T + k - 1);
-            }
-        } else {
-#pragma unroll
-            for (int v = 0; v < 3 * G; ++v) x[v] = __ldg(xk + v);
-            if (ov) {
-#pragma unroll
-                for (int v = 0; v < 3 * G; ++v) xp[v] = __ldg(xq + v);
-                gp = load_map(gmaps + (int64_t)q * T + k - 1);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < G; ++u) apply(gk, x + 3 * u, y + 3 * u);
-        if (ov) {
-#pragma unroll
-            for (int u = 0; u < G; ++u) {
-                float y1[3];
-                apply(gp, xp + 3 * u, y1);
-#pragma unroll
-                for (int d = 0; d < 3; ++d) y[3 * u + d] = 0.5f * (y1[d] + y[3 * u + d]);
-            }
-        }
-        float *dst = chain + ((int64_t)pair * L + p) * 3;
-        if constexpr (G == 4) {
-#pragma unroll
-            for (int v = 0; v < 3; ++v) reinterpret_cast<float4 *>(dst)[v] = *reinterpret_cast<const float4 *>(y + 4 * v);
-        } else {
-#pragma unroll
-            for (int v = 0; v < 3 * G; ++v) dst[v] = y[v];
-        }
+        place_group<G, true>(coords, T, B, o, c, b, p, gmaps + (int64_t)q * T, chain + ((int64_t)pair * L + p) * 3);
     }
+}
+
+// The one-pass form for chains of at most kFusedMaxT tiles: one CTA of 128
+// threads per (chain, sample) pair, 7 CTAs per SM (72 registers, no spills),
+// so that 1036 pairs are resident at once.  Warp 0 computes the pair's maps into
+// shared memory (pair_maps), then all threads place its beads.
+constexpr int kFusedMaxT = 512;
+constexpr int kFusedThreads = 128;
+
+template <int G>
+__global__ void __launch_bounds__(kFusedThreads, 7) stitch_kernel(const float *__restrict__ coords, int T, int B, int o,
+                                                     float *__restrict__ chain, float *__restrict__ resid) {
+    extern __shared__ __align__(16) float sm[];    // [2][32][3o+1] bead staging, then [T] maps
+    Rigid *smaps = reinterpret_cast<Rigid *>(sm + 2 * 32 * (3 * o + 1));
+    const int64_t pair = blockIdx.x;
+    const int c = (int)(pair / B), b = (int)(pair - (int64_t)(pair / B) * B);
+    if (threadIdx.x < 32) pair_maps(coords, T, B, o, c, b, pair, sm, resid, smaps);
+    __syncthreads();
+    const int L = kN + (T - 1) * (kN - o);
+    float *dst = chain + pair * (int64_t)L * 3;
+    for (int g = threadIdx.x; g < L / G; g += blockDim.x)
+        place_group<G, false>(coords, T, B, o, c, b, g * G, smaps, dst + (int64_t)g * G * 3);
 }
 
 }  // namespace
@@ -386,13 +452,22 @@ cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, fl
     // T <= 65535 (checked with the tiling) keeps one pair's maps within the scratch
     const int64_t chunk = scratch == nullptr ? 0 : (int64_t)scratch_floats / per_pair;
     if (chunk < 1) return cudaErrorInvalidValue;
+    const bool vec = o % 4 == 0;
+    if (t.T <= kFusedMaxT) {
+        // 2 * 32 * (3o + 1) floats: a multiple of 16 bytes, so the maps that follow are aligned
+        const size_t smem = sizeof(float) * 2 * 32 * (3 * o + 1) + sizeof(Rigid) * (size_t)t.T;
+        if (vec)
+            stitch_kernel<4><<<(unsigned)pairs, kFusedThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
+        else
+            stitch_kernel<1><<<(unsigned)pairs, kFusedThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
+        return cudaGetLastError();
+    }
     Rigid *gmaps = reinterpret_cast<Rigid *>(scratch);
     for (int64_t p0 = 0; p0 < pairs; p0 += chunk) {
         const int64_t n = pairs - p0 < chunk ? pairs - p0 : chunk;
         const size_t smem = sizeof(float) * 2 * 32 * (3 * o + 1);
         stitch_align_kernel<<<(unsigned)n, 32, smem, st>>>(coords, t.T, t.B, o, p0, gmaps, resid);
         const int64_t beads = n * (kN + (int64_t)(t.T - 1) * (kN - o));
-        const bool vec = o % 4 == 0;
         int64_t blocks = ((vec ? beads / 4 : beads) + 255) / 256;
         if (blocks > 148LL * 64) blocks = 148LL * 64;
         if (vec)
