@@ -211,8 +211,11 @@ tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, co
  * first_step = S-1) and written back.  The noise is keyed by the step index
  * and the projection follows the steps counted from step S-1, so a run split
  * into parts (the state kept in maps in between, e.g. saved and restored as a
- * checkpoint) gives the same maps, bit for bit, as the whole run.  Errors as
- * tdm_ddim_run, plus TDM_EINVAL for a step range outside the schedule. */
+ * checkpoint) follows the whole run: its states equal the whole run's up to
+ * the float32 rounding of the state written at each cut, and its final maps
+ * (after step 0, which sets them from x0 and that step's own noise) are the
+ * same bit for bit.  Errors as tdm_ddim_run, plus TDM_EINVAL for a step range
+ * outside the schedule. */
 tdm_status tdm_ddim_run_steps(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w,
                               float s_c, float s_u, uint64_t seed, int32_t init_noise, int32_t first_step,
                               int32_t n_steps, const tdm_tiling *tiling, tdm_stream stream);

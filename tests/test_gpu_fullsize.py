@@ -53,8 +53,13 @@ def test_step_sweep_chain32_b100(tdm, eta):
         ref = closed_form_final(x0, sample_ids(1, 32, b_check, 100), wl.seed, wl.w, wl.s_c, wl.s_u, True)
         assert_maps_close(g[:, :, b_check], ref, TOL_MAP, f"S={S} closed form")
         if S == 50:
-            full = o_run(x0, osched.Schedule(S=S, eta=eta), wl.w, wl.s_c, wl.s_u, wl.seed, [int(b_check[0])], 100)
+            full, traj = o_run(x0, osched.Schedule(S=S, eta=eta), wl.w, wl.s_c, wl.s_u, wl.seed,
+                               [int(b_check[0])], 100, return_trajectory=True)
             assert_maps_close(g[:, :, b_check[:1]], full, TOL_MAP, f"S={S} oracle run")
+            # the state before the last step, which alone sets the final maps
+            tdm.ddim_run(sch, maps, dev(x0), wl.w, wl.s_c, wl.s_u, wl.seed, t, first_step=S - 1, n_steps=S - 1)
+            g = host(maps).reshape(1, 32, 100, 64, 64)
+            assert_maps_close(g[:, :, b_check[:1]], traj[S - 2], TOL_MAP, f"S={S} oracle run, {S - 1} steps")
 
 
 def test_genome_untiled_chunked(tdm):

@@ -197,8 +197,13 @@ def test_fused_equals_per_step_on_symmetric_start(tdm):
     x0 = synth.chain_x0(2, 1, 3)
     fused = _maps(t)
     tdm.ddim_run(sch, fused, dev(x0), 1.0, 0.1, 0.3, 8, t)
-    per = _gpu_per_step(tdm, sch, x0, t, 1.0, 0.1, 0.3, 8)[-1]
-    assert normwise(_as5(fused, t), per).max() < 2 * TOL_MAP
+    states = _gpu_per_step(tdm, sch, x0, t, 1.0, 0.1, 0.3, 8)
+    assert normwise(_as5(fused, t), states[-1]).max() < 2 * TOL_MAP
+    # and a state before the last step (which alone sets the final maps)
+    for m in (5, 24):
+        part = _maps(t)
+        tdm.ddim_run(sch, part, dev(x0), 1.0, 0.1, 0.3, 8, t, first_step=24, n_steps=m)
+        assert normwise(_as5(part, t), states[m - 1]).max() < 2 * TOL_MAP, m
 
 
 def test_fused_run_is_deterministic_and_shards_reproduce_it(tdm):
@@ -227,10 +232,15 @@ def test_chromosome_chain_full_size_sampled(tdm):
     maps = _maps(t)
     tdm.ddim_run(sch, maps, dev(x0), wl.w, wl.s_c, wl.s_u, wl.seed, t)
     g = maps.view(1, 32, 1000, 64, 64)
+    refs = {}
     for b in (0, 417, 999):
-        ref = o_run(x0, osched.Schedule(S=50), wl.w, wl.s_c, wl.s_u, wl.seed, [b], 1000)
-        assert_maps_close(host(g[:, :, b:b + 1]), ref, TOL_MAP, f"sample {b}")
+        refs[b] = o_run(x0, osched.Schedule(S=50), wl.w, wl.s_c, wl.s_u, wl.seed, [b], 1000, return_trajectory=True)
+        assert_maps_close(host(g[:, :, b:b + 1]), refs[b][0], TOL_MAP, f"sample {b}")
     assert torch.isfinite(g).all()
+    # the same launch stopped before the last step, which alone sets the final maps
+    tdm.ddim_run(sch, maps, dev(x0), wl.w, wl.s_c, wl.s_u, wl.seed, t, first_step=49, n_steps=49)
+    for b in (0, 417, 999):
+        assert_maps_close(host(g[:, :, b:b + 1]), refs[b][1][48], TOL_MAP, f"sample {b}, 49 steps")
 
 
 def test_invalid_arguments_are_rejected(tdm):
