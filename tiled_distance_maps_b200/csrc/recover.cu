@@ -5,13 +5,16 @@
 // reading used is classical MDS: B = -1/2 J (D*D) J, the top three eigenpairs,
 // x_k = v_k sqrt(max(l_k, 0)).
 //
-// Per map, one warp stages D in shared memory and forms B in place.  The top eigenpairs come from subspace iteration on three
-// vectors with a Rayleigh-Ritz step (a 3 x 3 Jacobi eigen-solve) every
-// iteration, stopping when the residual of the three Ritz pairs is below
-// kTol * |l_1|.  The start basis is the three columns of B with the largest
-// diagonal entries (the points farthest from the centroid): for an exact
-// Euclidean map they already span the answer.  Row l of B stays in registers
-// for the products; row l+32 is read from shared memory.
+// Per map, one warp stages D in shared memory by 16-byte asynchronous copies
+// (the warp's next map is meanwhile brought into L2 by one bulk prefetch, so
+// those copies wait on L2 rather than DRAM) and forms B in place.  The top
+// eigenpairs come from subspace iteration on three vectors with a
+// Rayleigh-Ritz step (a 3 x 3 Jacobi eigen-solve) every iteration, stopping
+// when the residual of the three Ritz pairs is below kTol * |l_1|.  The start
+// basis is the three columns of B with the largest diagonal entries (the
+// points farthest from the centroid): for an exact Euclidean map they already
+// span the answer.  Row l of B stays in registers for the products; row l+32
+// is read from shared memory.
 #include "common.cuh"
 
 namespace tdm {
@@ -168,14 +171,24 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
 
     for (int64_t m = (int64_t)blockIdx.x * kMdsWarps + warp; m < n; m += (int64_t)gridDim.x * kMdsWarps) {
         const float *D = maps + m * kMapFloats;
-        // 16 loads of the map in flight per lane before their stores (8 left
-        // 2.6 % more time exposed to the load latency; 32 cost more registers)
-#pragma unroll 16
-        for (int it = 0; it < 32; ++it) {
-            const int idx = it * 32 + lane;
-            const int row = idx >> 4, c4 = (idx & 15) << 2;
-            *reinterpret_cast<float4 *>(sD + row * kLd + c4) =
-                __ldcs(reinterpret_cast<const float4 *>(D + row * kN + c4));
+        {   // the warp's next map into L2 while this one is processed
+            const int64_t mn = m + (int64_t)gridDim.x * kMdsWarps;
+            if (lane == 0 && mn < n)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(maps + mn * kMapFloats),
+                             "r"((unsigned)(kMapFloats * sizeof(float)))
+                             : "memory");
+        }
+        {   // the map into shared memory by 16-byte asynchronous copies, all in flight at once
+            const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(sD));
+#pragma unroll
+            for (int it = 0; it < 32; ++it) {
+                const int idx = it * 32 + lane;
+                const int row = idx >> 4, c4 = (idx & 15) << 2;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + 4u * (row * kLd + c4)),
+                             "l"(D + row * kN + c4)
+                             : "memory");
+            }
+            asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
         }
         __syncwarp();
 
@@ -369,7 +382,7 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
             const float2 cy = reinterpret_cast<const float2 *>(sc + kN)[lane];
             const float2 cz = reinterpret_cast<const float2 *>(sc + 2 * kN)[lane];
             float2 *out = reinterpret_cast<float2 *>(dist + m * kMapFloats) + lane;
-#pragma unroll 4
+#pragma unroll 8
             for (int row = 0; row < kN; ++row) {
                 const float xi = sc[row], yi = sc[kN + row], zi = sc[2 * kN + row];
                 float2 d;
