@@ -193,34 +193,27 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         __syncwarp();
 
         // e_ij = D_ij + D_ji (twice the symmetric part); S = (e/2)^2, so
-        // B = -1/2 J S J = -1/8 J (e*e) J.  Each unordered pair {v, w} is
-        // read and written by one lane only (virtual lane v in {l, l+32} takes
-        // w = v + k mod 64 for k = 0..32, and k = 32 only for v < 32), so e*e
-        // replaces D at (v, w) and (w, v) with no barrier between the reads
-        // and the writes; banks (5 l + k) and (5 l + 4 k) mod 32 are distinct
-        // over the lanes.
-#pragma unroll 3
-        for (int k = 0; k <= 32; ++k) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                if (k == 32 && h == 1) continue;
-                const int v = lane + 32 * h;
-                const int w = (v + k) & (kN - 1);
-                const float e = sD[v * kLd + w] + sD[w * kLd + v];
-                const float e2 = e * e;
-                sD[v * kLd + w] = e2;
-                sD[w * kLd + v] = e2;
-            }
-        }
-        __syncwarp();
-        // row means of e*e (lane: rows i0 and i1), grand mean
+        // B = -1/2 J S J = -1/8 J (e*e) J.  Lane l forms e*e of rows i0 and
+        // i1 in registers from row reads (float4) and column reads (lane l
+        // reads column l or l+32 of row j: consecutive words), all before any
+        // write, so no element is overwritten while another lane reads it.
+        float t0[kN], t1[kN];
         float rs0 = 0.0f, rs1 = 0.0f;
-#pragma unroll 4
+#pragma unroll
         for (int j4 = 0; j4 < kN / 4; ++j4) {
             const float4 a = *reinterpret_cast<const float4 *>(sD + i0 * kLd + 4 * j4);
             const float4 b = *reinterpret_cast<const float4 *>(sD + i1 * kLd + 4 * j4);
-            rs0 += (a.x + a.y) + (a.z + a.w);
-            rs1 += (b.x + b.y) + (b.z + b.w);
+            const float ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = 4 * j4 + u;
+                const float e0 = ra[u] + sD[j * kLd + i0], e1 = rb[u] + sD[j * kLd + i1];
+                t0[j] = e0 * e0;
+                t1[j] = e1 * e1;
+            }
+            // row sums in the order of a float4 pass over the rows
+            rs0 += (t0[4 * j4] + t0[4 * j4 + 1]) + (t0[4 * j4 + 2] + t0[4 * j4 + 3]);
+            rs1 += (t1[4 * j4] + t1[4 * j4 + 1]) + (t1[4 * j4 + 2] + t1[4 * j4 + 3]);
         }
         const float r0 = rs0 * (1.0f / kN), r1 = rs1 * (1.0f / kN);
         const float gm = wsum(r0 + r1) * (1.0f / kN);
@@ -232,24 +225,23 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         const float cs = -0.125f * scale;
         sR[i0] = r0;
         sR[i1] = r1;
-        __syncwarp();
-        // double centring in place, row by row: B_ij = cs (e2_ij - r_i - r_j + g);
-        // row i0 of B is also kept in registers for the products
+        __syncwarp();    // every lane's reads of D are done: rows of B may replace it
+        // double centring: B_ij = cs (e2_ij - r_i - r_j + g); row i0 of B is
+        // also kept in registers for the products
         const float g0 = gm - r0, g1 = gm - r1;
-        float b0[kN];
+        float *b0 = t0;
 #pragma unroll
         for (int j4 = 0; j4 < kN / 4; ++j4) {
             const float4 rj = *reinterpret_cast<const float4 *>(sR + 4 * j4);
-            float4 a = *reinterpret_cast<const float4 *>(sD + i0 * kLd + 4 * j4);
-            float4 b = *reinterpret_cast<const float4 *>(sD + i1 * kLd + 4 * j4);
-            a.x = cs * ((a.x + g0) - rj.x);
-            a.y = cs * ((a.y + g0) - rj.y);
-            a.z = cs * ((a.z + g0) - rj.z);
-            a.w = cs * ((a.w + g0) - rj.w);
-            b.x = cs * ((b.x + g1) - rj.x);
-            b.y = cs * ((b.y + g1) - rj.y);
-            b.z = cs * ((b.z + g1) - rj.z);
-            b.w = cs * ((b.w + g1) - rj.w);
+            float4 a, b;
+            a.x = cs * ((t0[4 * j4] + g0) - rj.x);
+            a.y = cs * ((t0[4 * j4 + 1] + g0) - rj.y);
+            a.z = cs * ((t0[4 * j4 + 2] + g0) - rj.z);
+            a.w = cs * ((t0[4 * j4 + 3] + g0) - rj.w);
+            b.x = cs * ((t1[4 * j4] + g1) - rj.x);
+            b.y = cs * ((t1[4 * j4 + 1] + g1) - rj.y);
+            b.z = cs * ((t1[4 * j4 + 2] + g1) - rj.z);
+            b.w = cs * ((t1[4 * j4 + 3] + g1) - rj.w);
             b0[4 * j4] = a.x;
             b0[4 * j4 + 1] = a.y;
             b0[4 * j4 + 2] = a.z;
