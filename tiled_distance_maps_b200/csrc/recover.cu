@@ -6,8 +6,9 @@
 // x_k = v_k sqrt(max(l_k, 0)).
 //
 // Per map, one warp stages D in shared memory by 16-byte asynchronous copies
-// (the warp's next map is meanwhile brought into L2 by one bulk prefetch, so
-// those copies wait on L2 rather than DRAM) and forms B in place.  The top
+// (the warp's next map is brought into L2 by one bulk prefetch issued when the
+// current map's eigen-solve is done, so those copies wait on L2 rather than
+// DRAM) and forms B.  The top
 // eigenpairs come from subspace iteration on three vectors with a
 // Rayleigh-Ritz step (a 3 x 3 Jacobi eigen-solve) every iteration, stopping
 // when the residual of the three Ritz pairs is below kTol * |l_1|.  The start
@@ -171,13 +172,6 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
 
     for (int64_t m = (int64_t)blockIdx.x * kMdsWarps + warp; m < n; m += (int64_t)gridDim.x * kMdsWarps) {
         const float *D = maps + m * kMapFloats;
-        {   // the warp's next map into L2 while this one is processed
-            const int64_t mn = m + (int64_t)gridDim.x * kMdsWarps;
-            if (lane == 0 && mn < n)
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(maps + mn * kMapFloats),
-                             "r"((unsigned)(kMapFloats * sizeof(float)))
-                             : "memory");
-        }
         {   // the map into shared memory by 16-byte asynchronous copies, all in flight at once
             const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(sD));
 #pragma unroll
@@ -344,6 +338,15 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
             sV01[i1] = make_float2(v1[0], v1[1]);
             sV2[i0] = v0[2];
             sV2[i1] = v1[2];
+        }
+        {   // the warp's next map into L2 while this one's coordinates and
+            // distances are written (issued at the start of the map, or before
+            // the eigen-solve, it measured slower)
+            const int64_t mn = m + (int64_t)gridDim.x * kMdsWarps;
+            if (lane == 0 && mn < n)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(maps + mn * kMapFloats),
+                             "r"((unsigned)(kMapFloats * sizeof(float)))
+                             : "memory");
         }
         if (!conv && lane == 0) atomicOr(flags, (uint32_t)TDM_FLAG_MDS_NOT_CONVERGED);
 
