@@ -19,6 +19,16 @@ mdpi.com/2079-9292/15/13/2750):
   mds            -- classical MDS (the distance-geometry initialisation of
                     §3.1) and pairwise-distance reconstruction
 
+and, beyond that path:
+
+  schedule       -- the cosine alphas-bar table (§4.3.2 names a cosine
+                    schedule; Nichol & Dhariwal 2021)
+  ddim           -- the DDPM ancestral step (§5.1.2), written separately
+  drift          -- the non-overlap drift of a synchronisation sweep (§5.7)
+  stitch         -- Kabsch stitching of tile coordinates (§4.3.2, §5.5 Fig. 4)
+  refine         -- SMACOF coordinate refinement (§3.1: "followed by
+                    coordinate refinement")  [reading]
+
 Every function is float64 and follows the definition or the algorithm's steps
 as written; readings of passages that the pages leave open are stated in each
 function.  Parity status: every function here is pinned by a CPU test against
