@@ -312,6 +312,8 @@ def run_ours(args, rank, world, local_rank):
             step()
         torch.cuda.synchronize()
         flags = tdm.ctx_sync(ctx)
+        # the measured FMA rate, the other denominator of the ALU rooflines
+        fma_rate = tdm.fma_rate(ctx)
         barrier()
         torch.cuda.synchronize()
         clocks.mark_start()
@@ -466,6 +468,8 @@ def run_ours(args, rank, world, local_rank):
                          "peak": peak / 1e12, "unit": "Tops/s", "frac": achieved / peak,
                          "traffic": profiled_traffic("ddim_run_kernel_chain32_b1000_cfg.md", RUN_SOURCES),
                          "peak_kind": "derived: 148 SMs x 128 lanes x max SM clock",
+                         "peak_measured": fma_rate / 1e12, "frac_measured": achieved / fma_rate,
+                         "peak_measured_kind": "tdm_fma_rate: independent fmaf chains, 8 CTAs x 256 threads per SM",
                          "ms_per_launch": run_avg_ms,
                          "ops_per_launch": ops},
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"], "samples": clk["samples"]},
@@ -483,7 +487,7 @@ def run_ours(args, rank, world, local_rank):
                               "frac": n_maps * 4 * 4096 * 4 / (step_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
                               "note": "one DDIM step of 32,000 maps, CFG w=1: read x, eps_c, eps_u, write x "
                                       "(64 KiB per map); timed separately from the step above"},
-            "next_rows": _next_rows(nx, n_maps, B, T, L, peak, float(peaks["hbm_gbs"])),
+            "next_rows": _next_rows(nx, n_maps, B, T, L, peak, float(peaks["hbm_gbs"]), fma_rate),
             "small_case": nx["small_case"],
             "mds_not_converged": bool(flags & tdm.FLAG_MDS_NOT_CONVERGED),
             "peaks": kind,
@@ -572,7 +576,7 @@ def _time_flushed(fn, stream, flush, n: int = 10) -> float:
     return float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n)]))
 
 
-def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
+def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs, fma_rate=None):
     """Roofline lines of the kernels beyond the step (rank 0, this GPU)."""
     ops = n_maps * REFINE_ITERATIONS * 64 * 64 * OPS_GUTTMAN_PAIR
     st_bytes = n_maps * 192 * 4 + B * L * 3 * 4 + B * (T - 1) * 4
@@ -583,6 +587,7 @@ def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs):
                           "ms_per_launch": nx["refine_smacof"], "ops_per_launch": ops,
                           "achieved": ops / (nx["refine_smacof"] / 1e3) / 1e12, "peak": alu_peak / 1e12,
                           "unit": "Tops/s", "frac": ops / (nx["refine_smacof"] / 1e3) / alu_peak,
+                          "frac_measured": (ops / (nx["refine_smacof"] / 1e3) / fma_rate) if fma_rate else None,
                           "traffic": profiled_traffic("refine_kernel_chain32_b1000_cfg.md", REFINE_SOURCES),
                           "note": f"{n_maps} coordinate sets x {REFINE_ITERATIONS} Guttman transforms, "
                                   f"{OPS_GUTTMAN_PAIR} lane-ops per ordered pair, plus the final stress"},

@@ -128,6 +128,16 @@ tdm_status tdm_ctx_sync(tdm_ctx *ctx, tdm_stream stream, uint32_t *flags_out);
  * misaligned buf with n > 0). */
 tdm_status tdm_scan_nonfinite(tdm_ctx *ctx, const float *buf, int64_t n, tdm_stream stream);
 
+/* Diagnostics: the device's float32 FMA rate, measured by two launches of a
+ * kernel in which every thread of 8 CTAs x 256 threads per SM runs 8
+ * independent fmaf chains, the second launch timed with CUDA events on
+ * `stream`.  *fma_per_s receives fused multiply-adds per second, one per
+ * lane and instruction: the measured denominator of the ALU rooflines (in
+ * theory one per CUDA-core lane per clock).  The kernel writes nothing
+ * (its guarded store into the context's scratch never fires).  Synchronises
+ * `stream`.  Errors: TDM_EINVAL (NULL ctx or output), TDM_ECUDA. */
+tdm_status tdm_fma_rate(tdm_ctx *ctx, double *fma_per_s, tdm_stream stream);
+
 /* The cosine alphas-bar table of Nichol & Dhariwal, "Improved Denoising
  * Diffusion Probabilistic Models" (2021, section 3.2), for passing to
  * tdm_init_schedule as alphas_bar_opt: alphas_bar(t) = f(t) / f(0),

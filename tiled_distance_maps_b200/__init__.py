@@ -69,6 +69,7 @@ _SIGS = {
     "tdm_nonoverlap_drift": (_i32, [_vp, _vp, _vp, _P(CTiling), _vp, _vp, _vp]),
     "tdm_cosine_alphas_bar": (_i32, [_i32, _f64, _vp]),
     "tdm_scan_nonfinite": (_i32, [_vp, _vp, _i64, _vp]),
+    "tdm_fma_rate": (_i32, [_vp, ctypes.POINTER(_f64), _vp]),
     "tdm_mds_reconstruct": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -492,3 +493,13 @@ def scan_nonfinite(buf, ctx: Context | None = None):
     ctx = ctx or context(buf.device.index)
     ctx.check(_lib.tdm_scan_nonfinite(ctx.handle, _uptr(buf, "buf", ctx, torch.float32), int(buf.numel()),
                                       _stream(ctx)))
+
+
+def fma_rate(ctx: Context | None = None) -> float:
+    """The device's measured float32 FMA rate in FMAs per second, the
+    denominator of the ALU rooflines (see tdm_fma_rate); synchronises the
+    current stream."""
+    ctx = ctx or context()
+    out = _f64(0.0)
+    ctx.check(_lib.tdm_fma_rate(ctx.handle, _c.byref(out), _stream(ctx)))
+    return float(out.value)

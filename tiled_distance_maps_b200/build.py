@@ -21,7 +21,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtdm.so")
-SOURCES = ["api.cpp", "sampler.cu", "seam.cu", "recover.cu", "refine.cu", "drift.cu", "scan.cu", "stitch.cu", "noalloc.cu"]
+SOURCES = ["api.cpp", "sampler.cu", "seam.cu", "recover.cu", "refine.cu", "drift.cu", "scan.cu", "stitch.cu", "noalloc.cu",
+           "peak.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

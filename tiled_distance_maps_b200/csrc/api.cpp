@@ -190,6 +190,32 @@ tdm_status tdm_scan_nonfinite(tdm_ctx *ctx, const float *buf, int64_t n, tdm_str
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "scan launch");
 }
 
+tdm_status tdm_fma_rate(tdm_ctx *ctx, double *fma_per_s, tdm_stream stream) {
+    NvtxRange nvtx_range_("tdm_fma_rate");
+    if (ctx == nullptr) return TDM_EINVAL;
+    if (fma_per_s == nullptr) return fail(ctx, TDM_EINVAL, "fma_rate: output is NULL");
+    DeviceScope ds(ctx->device);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaEvent_t ev[2] = {nullptr, nullptr};
+    cudaError_t e = cudaEventCreate(&ev[0]);
+    if (e == cudaSuccess) e = cudaEventCreate(&ev[1]);
+    double fmas = 0.0;
+    // one short launch to reach full clocks, then the timed one
+    if (e == cudaSuccess) e = tdm::launch_fma_rate(ctx->d_scratch, (int64_t)ctx->scratch_floats, 256, st, &fmas);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[0], st);
+    if (e == cudaSuccess) e = tdm::launch_fma_rate(ctx->d_scratch, (int64_t)ctx->scratch_floats, 4096, st, &fmas);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[1], st);
+    if (e == cudaSuccess) e = cudaEventSynchronize(ev[1]);
+    float ms = 0.0f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, ev[0], ev[1]);
+    if (ev[0] != nullptr) cudaEventDestroy(ev[0]);
+    if (ev[1] != nullptr) cudaEventDestroy(ev[1]);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "fma_rate");
+    if (!(ms > 0.0f)) return fail(ctx, TDM_ECUDA, "fma_rate: no elapsed time");
+    *fma_per_s = fmas / ((double)ms * 1e-3);
+    return TDM_OK;
+}
+
 // ---- schedule -----------------------------------------------------------------------
 
 tdm_status tdm_cosine_alphas_bar(int32_t T_train, double s, double *alphas_bar_out) {

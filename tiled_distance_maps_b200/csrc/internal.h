@@ -89,6 +89,7 @@ std::vector<uint32_t> build_run_plan(int T, int overlap);
 int seam_chunks(int64_t n_seams, int B);
 int drift_chunks(int64_t tiles, int B);
 cudaError_t launch_scan_nonfinite(const float *buf, int64_t n, uint32_t *flags, cudaStream_t st);
+cudaError_t launch_fma_rate(float *sink, int64_t sink_floats, int iters, cudaStream_t st, double *fmas);
 cudaError_t launch_drift(const float *S, const float *V, const Tiling &t, float *scratch, int chunks,
                          float *tile_sums, float *drift, cudaStream_t st);
 
