@@ -620,18 +620,29 @@ def _seam_chunks(n_seams, B):
     return max(1, min(ch, -(-B // 8)))
 
 
-def _events_ms(fn, reps: int = 1) -> float:
-    """Device ms of ``reps`` back-to-back calls of ``fn`` (one untimed first)."""
+def _median_ms(fn, reps: int = 10) -> float:
+    """Median device ms of ``reps`` calls of ``fn``, each timed on its own by
+    CUDA events (one untimed call first)."""
     import torch
     fn()
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(reps):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+    for i in range(reps):
+        ev[2 * i].record()
         fn()
-    b.record()
+        ev[2 * i + 1].record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / reps
+    return float(np.median([ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(reps)]))
+
+
+def _over_seeds(values: dict) -> dict:
+    """Mean and sample standard deviation of per-seed values."""
+    v = np.array(list(values.values()), dtype=np.float64)
+    return {"mean": float(v.mean()), "sd": float(v.std(ddof=1)) if v.size > 1 else 0.0,
+            "per_seed": {str(k): float(x) for k, x in values.items()}}
+
+
+SEEDS = (0, 1, 2)
 
 
 def run_configs(args) -> int:
@@ -668,13 +679,21 @@ def run_configs(args) -> int:
     maps, coords, rec = (torch.empty(n * k, device=dev) for k in (4096, 192, 4096))
     disc = torch.empty(wl.T - 1, device=dev)
 
-    def step2():
-        tdm.ddim_run(sch, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, t, ctx=ctx)
-        tdm.mds_reconstruct(maps, n, coords, rec, ctx=ctx)
-        tdm.seam_discrepancy(rec, t, disc, ctx=ctx)
-    ms = _events_ms(step2, 5)
+    per_seed = {}
+    for seed in SEEDS:
+        x0 = torch.from_numpy(synth.chain_x0(seed, 1, wl.T, sigma=wl.sigma)).to(dev)
+
+        def step2():
+            tdm.ddim_run(sch, maps, x0, wl.w, wl.s_c, wl.s_u, seed, t, ctx=ctx)
+            tdm.mds_reconstruct(maps, n, coords, rec, ctx=ctx)
+            tdm.seam_discrepancy(rec, t, disc, ctx=ctx)
+        per_seed[seed] = n * wl.S / (_median_ms(step2, 10) / 1e3)
+    st2 = _over_seeds(per_seed)
     lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
-                  "value": n * wl.S / (ms / 1e3), "ms_per_step": ms, "bound": "alu (fused run)"})
+                  "value": st2["mean"], "sd": st2["sd"], "per_seed": st2["per_seed"],
+                  "ms_per_step": n * wl.S / st2["mean"] * 1e3, "bound": "alu (fused run)",
+                  "note": "per seed (noise seed and x0 walk seed 0, 1, 2): the median of 10 steps, each timed by "
+                          "CUDA events; value and sd over the seeds"})
     del maps, coords, rec
 
     # cfg3: the step sweep on the 32-tile x 100-sample chain, w = 0
@@ -687,14 +706,21 @@ def run_configs(args) -> int:
     for eta in wl.extra["eta"]:
         for S in wl.extra["S"]:
             sch = tdm.Schedule(S, eta, ctx=ctx)
-            ms = _events_ms(lambda: tdm.ddim_run(sch, maps, x0, wl.w, wl.s_c, wl.s_u, wl.seed, t, ctx=ctx), 3)
+            rates = {}
+            for seed in SEEDS:
+                x0s = torch.from_numpy(synth.chain_x0(seed, 1, wl.T)).to(dev)
+                ms = _median_ms(lambda: tdm.ddim_run(sch, maps, x0s, wl.w, wl.s_c, wl.s_u, seed, t, ctx=ctx), 10)
+                rates[seed] = n * S / (ms / 1e3)
+            st3 = _over_seeds(rates)
             ns = 1 + (1 if eta > 0 else 0)
             ops = ops_per_map_step(ns) * n * S + QUADS_PER_MAP * n * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR)
-            sweep.append({"S": S, "eta": eta, "ms": ms, "map_steps_per_s": n * S / (ms / 1e3),
+            ms = n * S / st3["mean"] * 1e3
+            sweep.append({"S": S, "eta": eta, "ms": ms, "map_steps_per_s": st3["mean"], "sd": st3["sd"],
                           "alu_frac": ops / (ms / 1e3) / alu_peak})
     lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
                   "value": sum(x["map_steps_per_s"] for x in sweep) / len(sweep), "runs": sweep,
-                  "note": "value: mean over the 10 runs; alu_frac against the derived lane-op peak"})
+                  "note": "per run: the mean over seeds 0, 1, 2 of the median of 10 timed runs, and its sd; value: "
+                          "the mean over the 10 runs; alu_frac against the derived lane-op peak"})
     del maps
 
     # cfg4: 2658 regions x {w=0, w=1} x 256 samples, untiled, in chunks of 2^16 maps
@@ -703,40 +729,52 @@ def run_configs(args) -> int:
     chunk_regions = wl.extra["chunk_maps"] // B
     sch = tdm.Schedule(S, ctx=ctx)
     maps = torch.empty(chunk_regions * B * 4096, device=dev)
-    total_ms, total_ops = 0.0, 0
-    for gi, w in enumerate(wl.extra["w"]):
-        for r0 in range(0, R, chunk_regions):
-            nr = min(chunk_regions, R - r0)
-            x0 = torch.from_numpy(synth.region_x0(wl.seed, np.arange(r0, r0 + nr))).to(dev)
-            tt = tdm.Tiling(C=nr, T=1, B=B, overlap=0, sync_every=0, sample_id_base=gi * R * B + r0 * B)
-            total_ms += _events_ms(lambda: tdm.ddim_run(sch, maps, x0, w, wl.s_c, wl.s_u, wl.seed, tt, ctx=ctx))
-            ns = 1 + (1 if w != 0 else 0)
-            total_ops += ops_per_map_step(ns) * nr * B * S + QUADS_PER_MAP * nr * B * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR)
     steps4 = 2 * R * B * S
+    rates, dev_ms = {}, {}
+    for seed in SEEDS:
+        total_ms, total_ops = 0.0, 0
+        for gi, w in enumerate(wl.extra["w"]):
+            for r0 in range(0, R, chunk_regions):
+                nr = min(chunk_regions, R - r0)
+                x0 = torch.from_numpy(synth.region_x0(seed, np.arange(r0, r0 + nr))).to(dev)
+                tt = tdm.Tiling(C=nr, T=1, B=B, overlap=0, sync_every=0, sample_id_base=gi * R * B + r0 * B)
+                total_ms += _median_ms(lambda: tdm.ddim_run(sch, maps, x0, w, wl.s_c, wl.s_u, seed, tt, ctx=ctx), 10)
+                ns = 1 + (1 if w != 0 else 0)
+                total_ops += (ops_per_map_step(ns) * nr * B * S
+                              + QUADS_PER_MAP * nr * B * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR))
+        rates[seed], dev_ms[seed] = steps4 / (total_ms / 1e3), total_ms
+    st4 = _over_seeds(rates)
     lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
-                  "value": steps4 / (total_ms / 1e3), "device_ms": total_ms,
-                  "alu_frac": total_ops / (total_ms / 1e3) / alu_peak,
-                  "note": "1,360,896 trajectories in 22 chunks; the fused runs' device time summed"})
+                  "value": st4["mean"], "sd": st4["sd"], "per_seed": st4["per_seed"],
+                  "device_ms": float(np.mean(list(dev_ms.values()))),
+                  "alu_frac": total_ops / (steps4 / st4["mean"]) / alu_peak,
+                  "note": "1,360,896 trajectories in 22 chunks per guidance setting; per seed (0, 1, 2) the fused "
+                          "runs' device time summed over the chunks, each chunk the median of 10 timed runs"})
     del maps
 
     # cfg5: 1,000,000 noisy point-cloud maps: MDS + reconstruction, Eq. (6) over 31,250 x 32
     n = 1_000_000
     maps5 = torch.empty(n * 4096, device=dev)
-    g = torch.Generator(device=dev)
-    g.manual_seed(5)
-    for m0 in range(0, n, 100_000):
-        k = min(100_000, n - m0)
-        sig = torch.rand(k, 1, 1, device=dev, generator=g) * 9.0 + 1.0
-        pts = torch.randn(k, 64, 3, device=dev, generator=g) * sig
-        d = torch.cdist(pts, pts)
-        z = torch.triu(torch.randn(k, 64, 64, device=dev, generator=g), 1)
-        maps5[m0 * 4096:(m0 + k) * 4096] = (d * (1.0 + 0.01 * (z + z.transpose(1, 2)))).reshape(-1)
-        del sig, pts, d, z
     coords5, rec5 = torch.empty(n * 192, device=dev), torch.empty(n * 4096, device=dev)
     t5 = tdm.Tiling(C=31250, T=32, B=1, overlap=12, sync_every=0)
     disc5 = torch.empty(31250 * 31, device=dev)
-    ms_mds = _events_ms(lambda: tdm.mds_reconstruct(maps5, n, coords5, rec5, ctx=ctx))
-    ms_seam = _events_ms(lambda: tdm.seam_discrepancy(rec5, t5, disc5, ctx=ctx))
+    mds_ms, seam_ms = {}, {}
+    for seed in SEEDS:
+        g = torch.Generator(device=dev)
+        g.manual_seed(5 + seed)
+        for m0 in range(0, n, 100_000):
+            k = min(100_000, n - m0)
+            sig = torch.rand(k, 1, 1, device=dev, generator=g) * 9.0 + 1.0
+            pts = torch.randn(k, 64, 3, device=dev, generator=g) * sig
+            d = torch.cdist(pts, pts)
+            z = torch.triu(torch.randn(k, 64, 64, device=dev, generator=g), 1)
+            maps5[m0 * 4096:(m0 + k) * 4096] = (d * (1.0 + 0.01 * (z + z.transpose(1, 2)))).reshape(-1)
+            del sig, pts, d, z
+        mds_ms[seed] = _median_ms(lambda: tdm.mds_reconstruct(maps5, n, coords5, rec5, ctx=ctx), 10)
+        seam_ms[seed] = _median_ms(lambda: tdm.seam_discrepancy(rec5, t5, disc5, ctx=ctx), 10)
+    st5 = _over_seeds({k: n / ((mds_ms[k] + seam_ms[k]) / 1e3) for k in SEEDS})
+    ms_mds = float(np.mean(list(mds_ms.values())))
+    ms_seam = float(np.mean(list(seam_ms.values())))
     flags = tdm.ctx_sync(ctx)
     from oracle import mds as omds
     sample = maps5[:16 * 4096].view(16, 64, 64).cpu().numpy().astype(np.float64)
@@ -745,10 +783,12 @@ def run_configs(args) -> int:
     omds.pairwise_distances(Xo)
     dt = time.perf_counter() - t0
     lines.append({"config": "recovery_1m", "metric": "maps/sec", "unit": "maps/s",
-                  "value": n / ((ms_mds + ms_seam) / 1e3), "mds_reconstruct_ms": ms_mds, "seam_ms": ms_seam,
+                  "value": st5["mean"], "sd": st5["sd"], "per_seed": st5["per_seed"],
+                  "mds_reconstruct_ms": ms_mds, "seam_ms": ms_seam,
                   "hbm_frac_mds_reconstruct": n * (2 * 16384 + 768) / (ms_mds / 1e3) / 1e9 / float(peaks["hbm_gbs"]),
                   "oracle_maps_per_s_1core": 16 / dt, "mds_not_converged": bool(flags & tdm.FLAG_MDS_NOT_CONVERGED),
-                  "note": "inputs drawn on the device by torch for timing only"})
+                  "note": "inputs drawn on the device by torch for timing only (generator seeds 5, 6, 7); per "
+                          "seed the medians of 10 timed calls; value and sd over the seeds"})
     for line in lines:
         print(json.dumps(line), flush=True)
     return 0
