@@ -717,7 +717,17 @@ def run_configs(args) -> int:
             ms = n * S / st3["mean"] * 1e3
             sweep.append({"S": S, "eta": eta, "ms": ms, "map_steps_per_s": st3["mean"], "sd": st3["sd"],
                           "alu_frac": ops / (ms / 1e3) / alu_peak})
+    # the oracle on fixed subsets, extrapolated linearly (trajectories are independent)
+    from oracle import schedule as osched
+    from oracle.ddim import ddim_run as o_run
+    oracle3 = {}
+    for S, nb in ((50, 4), (1000, 1)):
+        x0h = synth.chain_x0(0, 1, wl.T)
+        t0 = time.perf_counter()
+        o_run(x0h, osched.Schedule(S=S, eta=0.0), wl.w, wl.s_c, wl.s_u, 0, np.arange(nb), wl.B)
+        oracle3[f"S={S}"] = wl.T * nb * S / (time.perf_counter() - t0)
     lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
+                  "oracle_map_steps_per_s_1core": oracle3,
                   "value": sum(x["map_steps_per_s"] for x in sweep) / len(sweep), "runs": sweep,
                   "note": "per run: the mean over seeds 0, 1, 2 of the median of 10 timed runs, and its sd; value: "
                           "the mean over the 10 runs; alu_frac against the derived lane-op peak"})
@@ -744,9 +754,18 @@ def run_configs(args) -> int:
                               + QUADS_PER_MAP * nr * B * (OPS_PHILOX + 2 * OPS_BOX_MULLER_PAIR))
         rates[seed], dev_ms[seed] = steps4 / (total_ms / 1e3), total_ms
     st4 = _over_seeds(rates)
+    # the oracle on 512 trajectories (256 per guidance setting, 8 regions x 32 samples each)
+    from oracle import schedule as osched
+    from oracle.ddim import ddim_run as o_run
+    t0 = time.perf_counter()
+    for gi, w in enumerate(wl.extra["w"]):
+        x0h = synth.region_x0(0, np.arange(8))
+        o_run(x0h, osched.Schedule(S=S), w, wl.s_c, wl.s_u, 0, np.arange(32), B, sync_every=0,
+              sample_id_base=gi * R * B)
+    oracle4 = 512 * S / (time.perf_counter() - t0)
     lines.append({"config": wl.name, "metric": "map-denoise-steps/sec", "unit": "map-steps/s",
                   "value": st4["mean"], "sd": st4["sd"], "per_seed": st4["per_seed"],
-                  "device_ms": float(np.mean(list(dev_ms.values()))),
+                  "device_ms": float(np.mean(list(dev_ms.values()))), "oracle_map_steps_per_s_1core": oracle4,
                   "alu_frac": total_ops / (steps4 / st4["mean"]) / alu_peak,
                   "note": "1,360,896 trajectories in 22 chunks per guidance setting; per seed (0, 1, 2) the fused "
                           "runs' device time summed over the chunks, each chunk the median of 10 timed runs"})
