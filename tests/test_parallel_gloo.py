@@ -1,10 +1,13 @@
 """The multi-GPU host logic on CPU: world size 2 over gloo.
 
-Each rank takes its shard of the samples, runs the sampler and Eq. (6)'s
-overlap sums on it (the float64 oracle stands in for the kernels here, since
-the kernels need a GPU), all-reduces the sums and finalises.  The result must
-equal the unsplit run: the maps of each shard bit for bit, Eq. (6) to
-rounding.
+Each rank takes its shard of the samples through the product's
+``parallel.shard_tiling``, runs the sampler on it, and computes Eq. (6) through
+the product's ``parallel.sharded_seam_discrepancy`` (overlap sums, the
+``allreduce_sums`` all-reduce, finalisation).  The two GPU halves of that
+wrapper are replaced by the float64 oracle on CPU tensors, since the kernels
+need a GPU; the sharding and the collective are the product's own code.  The
+result must equal the unsplit run: the maps of each shard bit for bit, Eq. (6)
+to rounding.
 """
 import os
 import socket
@@ -41,19 +44,34 @@ def _worker(rank, world, port, q):
     import torch.distributed as dist
 
     import synth
+    import tiled_distance_maps_b200 as tdm
     from oracle import schedule, seam
     from oracle.ddim import ddim_run
+    from tiled_distance_maps_b200 import parallel
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         C, T, B_total = 2, 3, 6
-        b0, nb = shard_range(B_total, rank, world)
+        t = parallel.shard_tiling(tdm.Tiling(C=C, T=T, B=B_total, overlap=12), rank, world)
+        assert t.B_total == B_total
         x0 = synth.chain_x0(3, C, T)
-        out = ddim_run(x0, schedule.Schedule(S=4), 1.0, 0.1, 0.3, 11, np.arange(b0, b0 + nb), B_total)
-        sums = torch.from_numpy(seam.overlap_difference_sums(out))
-        dist.all_reduce(sums)
-        disc = seam.discrepancy_from_sums(sums.numpy(), B_total)
-        q.put((rank, b0, out, disc))
+        out = ddim_run(x0, schedule.Schedule(S=4), 1.0, 0.1, 0.3, 11,
+                       np.arange(t.b_offset, t.b_offset + t.B), B_total)
+
+        # the kernels' halves of the wrapper, on CPU tensors through the oracle
+        def overlap_sums(maps, tiling, sums, ctx=None):
+            sums.copy_(torch.from_numpy(seam.overlap_difference_sums(maps)).reshape(sums.shape))
+
+        def finalize(sums, tiling, o, ctx=None):
+            shape = (tiling.C, tiling.T - 1, tiling.overlap, tiling.overlap)
+            o.copy_(torch.from_numpy(seam.discrepancy_from_sums(sums.numpy().reshape(shape),
+                                                                 tiling.B_total)).reshape(o.shape))
+
+        tdm.seam_overlap_sums, tdm.seam_discrepancy_finalize = overlap_sums, finalize
+        sums = torch.empty(C * (T - 1) * 12 * 12, dtype=torch.float64)
+        disc = torch.empty(C * (T - 1), dtype=torch.float64)
+        parallel.sharded_seam_discrepancy(out, t, sums, disc)
+        q.put((rank, t.b_offset, out, disc.numpy().reshape(C, T - 1)))
     finally:
         dist.destroy_process_group()
 

@@ -8,6 +8,7 @@
 // tdm_seam_discrepancy_noalloc needs no context (creating one allocates) and
 // keeps the partial sums of the chunked reduction in a fixed array below, which
 // every GPU that loads this library holds until the process exits.
+#include <map>
 #include <mutex>
 
 #include "internal.h"
@@ -19,21 +20,29 @@ static __device__ __align__(256) float g_noalloc_scratch[TDM_NOALLOC_SCRATCH_FLO
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-float *g_scratch_addr[kMaxDevices] = {};
+std::map<int, float *> g_scratch_addr;    // device index -> address seen by the last uncaptured call
 
-// Device address of g_noalloc_scratch on the current device `dev`, looked up
-// on the first call for that device and cached.
-cudaError_t scratch_address(int dev, float **out) {
+// Device address of g_noalloc_scratch on the current device `dev`.  A call
+// outside stream capture looks it up again (cheap once the module is loaded),
+// so a device reset or another current context is followed; a call under
+// capture takes the address of the last uncaptured call on that device, and
+// fails when there was none (the lookup may load the module, which a capture
+// must not see).
+cudaError_t scratch_address(int dev, cudaStream_t st, float **out) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cap);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
         g_scratch_addr[dev] = static_cast<float *>(p);
     }
-    *out = g_scratch_addr[dev];
+    const auto it = g_scratch_addr.find(dev);
+    if (it == g_scratch_addr.end()) return cudaErrorStreamCaptureUnsupported;
+    *out = it->second;
     return cudaSuccess;
 }
 
@@ -65,19 +74,20 @@ extern "C" tdm_status tdm_seam_discrepancy_noalloc(const float *maps, const tdm_
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const double inv_b = 1.0 / (double)t.B;
     const int chunks = tdm::seam_chunks(n_seams, t.B);
+    const int64_t need = n_seams * chunks * (int64_t)t.overlap * t.overlap;
     cudaError_t e;
-    if (chunks <= 1) {
-        // one warp per seam over all samples: no partial sums, no scratch
+    if (chunks <= 1 || need > TDM_NOALLOC_SCRATCH_FLOATS) {
+        // one warp (or CTA) per seam over all samples: no partial sums, no
+        // scratch; also the form for requests whose partial sums would not
+        // fit the fixed array
         e = tdm::launch_seam_finalize(maps, t, 0, inv_b, out, st);
     } else {
-        const int64_t need = n_seams * chunks * (int64_t)t.overlap * t.overlap;
-        if (need > TDM_NOALLOC_SCRATCH_FLOATS) return TDM_EUNSUPPORTED;
         int dev = 0;
         e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return TDM_ECUDA;
-        if (dev < 0 || dev >= kMaxDevices) return TDM_EUNSUPPORTED;
         float *scratch = nullptr;
-        e = scratch_address(dev, &scratch);
+        e = scratch_address(dev, st, &scratch);
+        if (e == cudaErrorStreamCaptureUnsupported) return TDM_EUNSUPPORTED;
         if (e != cudaSuccess) return TDM_ECUDA;
         // every partial sum that the finalisation reads is written first by
         // the sums kernel, so nothing has to start at zero
