@@ -26,9 +26,9 @@
  *    Launch failures are reported as TDM_ECUDA.
  *  - Every pointer named "device" is device memory owned by the caller; it must
  *    be 16-byte aligned and hold contiguous row-major float32 data.  The library
- *    never frees caller memory and allocates only inside tdm_ctx_create,
- *    tdm_init_schedule and on the first use of a new tiling shape (a small
- *    lookup table, cached in the context).
+ *    never frees caller memory and allocates only inside tdm_ctx_create and
+ *    tdm_init_schedule; the compute entry points allocate nothing and make no
+ *    synchronous copy.
  *  - Beads per tile n is 64.  A map is 64 x 64 float32 (16 KiB).
  *  - Tiled maps are laid out [C][T][B][64][64]: chain c, tile k, sample b.
  *    Reference maps x0 are [C][T][64][64], shared by the B samples of a tile
@@ -71,7 +71,7 @@ typedef int32_t tdm_status;
 #define TDM_SCHED_COLS 8   /* tau_i, ab_t, ab_p, sigma_i, a_i, b_i, sqrt(ab_t), 1/sqrt(1-ab_t) */
 
 typedef void *tdm_stream;              /* a cudaStream_t */
-typedef struct tdm_ctx tdm_ctx;        /* opaque: device, status word, scratch, plan cache */
+typedef struct tdm_ctx tdm_ctx;        /* opaque: device, status word, scratch */
 typedef struct tdm_schedule tdm_schedule;  /* opaque: DDIM coefficient table */
 
 /* Shape of a tiled batch.  C chains of T tiles (T = 1: independent, untiled
@@ -97,12 +97,12 @@ typedef struct tdm_tiling {
 /* Creates a context on CUDA device `device` (allocates its status word and
  * scratch).  *out receives the handle.  Errors: TDM_EINVAL (out NULL or bad
  * device), TDM_ENOMEM, TDM_ECUDA.  The calls that keep intermediate results
- * in the scratch (tdm_seam_discrepancy, tdm_nonoverlap_drift,
- * tdm_kabsch_stitch) must not overlap on the GPU for one context: issue them
- * on one stream, or give each stream its own context.  Host threads may share
- * a context (its lane-plan cache is locked), but the message of
- * tdm_ctx_last_error is the context's last one, whichever thread failed: a
- * thread that reads messages should have its own context. */
+ * in the scratch (tdm_seam_discrepancy, tdm_seam_overlap_sums,
+ * tdm_nonoverlap_drift) must not overlap on the GPU for one context: issue
+ * them on one stream, or give each stream its own context.  Host threads may share
+ * a context, but the message of tdm_ctx_last_error is the context's last one,
+ * whichever thread failed: a thread that reads messages should have its own
+ * context. */
 tdm_status tdm_ctx_create(tdm_ctx **out, int32_t device);
 
 /* Frees everything the context owns.  NULL is ignored. */
@@ -230,6 +230,17 @@ tdm_status tdm_ddim_run_steps(tdm_ctx *ctx, const tdm_schedule *sched, float *ma
                               float s_c, float s_u, uint64_t seed, int32_t init_noise, int32_t first_step,
                               int32_t n_steps, const tdm_tiling *tiling, tdm_stream stream);
 
+/* Which folded-state quad each lane of the fused run holds (host only; a
+ * diagnostic for callers that inspect the launch, and the map that the kernel
+ * derives in-kernel from the warp and lane index, with no table in memory).
+ * out[w * 32 + l] (host, n >= 544 T entries) receives, for lane l of warp w of
+ * a chain-sample's 17 T warps, q | r << 4 | k << 10 | paired << 31: row quad
+ * (r, 4q .. 4q+3) of tile k.  A paired lane (l < 16) holds a quad of the
+ * overlap block of tile k that the projection averages with the quad of tile
+ * k+1 in lane l + 16 of the same warp.  overlap: a multiple of 4 in [4, 32]
+ * when T > 1 (ignored when T = 1).  Errors: TDM_EINVAL. */
+tdm_status tdm_fused_lane_map(int32_t T, int32_t overlap, uint32_t *out, int64_t n);
+
 /* Overlap-consistency projection, in place (ParaChromo §4.3.2, Algorithm 1):
  * for every chain c, seam k < T-1 and sample b, M = 0.5 * (right block of tile
  * k + left block of tile k+1), the blocks being rows/cols [64-o, 64) and
@@ -262,8 +273,7 @@ tdm_status tdm_refine_smacof(tdm_ctx *ctx, const float *maps, int64_t n_maps, fl
  * bead is the mean of its two aligned copies.  residual_out: device
  * [C][B][T-1] (may be NULL), the RMSD over the o beads of each seam after the
  * alignment, in the coordinates' units.  Needs overlap >= 3 when T > 1.
- * The tiles' maps go through context scratch in chunks of (chain, sample)
- * pairs. */
+ * One pass over the coordinates for chains of any length; no scratch. */
 tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling *tiling, float *chain_out,
                              float *residual_out, tdm_stream stream);
 
@@ -345,15 +355,28 @@ tdm_status tdm_nonoverlap_drift(tdm_ctx *ctx, const float *maps, const float *re
  * allocator, or a pipeline that cannot afford the synchronisation that
  * cudaMalloc/cudaFree may imply.  It needs no tdm_ctx (creating one allocates).
  *
- * Computes exactly what tdm_seam_discrepancy computes (out: device [C][T-1];
- * maps: device [C][T][B][64][64]; both caller-owned, 16-byte aligned), on the
- * caller's current CUDA device and stream, and calls no cudaMalloc, cudaFree or
- * allocating routine.  When the samples of a seam are split into chunks, the
- * partial sums live in one fixed device array of TDM_NOALLOC_SCRATCH_FLOATS
- * floats (1 MiB) compiled into the library: every GPU that loads the library
- * holds it until the process exits.  The first call that needs it on a device
- * looks up its device address (cudaGetSymbolAddress) and caches it; make that
- * first call before any stream capture.
+ * Computes the seam discrepancy of Eq. (6) as tdm_seam_discrepancy does (out:
+ * device [C][T-1]; maps: device [C][T][B][64][64]; both caller-owned, 16-byte
+ * aligned), on the caller's current CUDA device and stream, and calls no
+ * cudaMalloc, cudaFree or allocating routine.  The result agrees with
+ * tdm_seam_discrepancy up to the float32 order of the sums.  When the samples
+ * of a seam are split into chunks, the partial sums live in one fixed device
+ * array of TDM_NOALLOC_SCRATCH_FLOATS floats (1 MiB) compiled into the
+ * library: every GPU that loads the library holds it until the process exits.
+ * Requests whose partial sums would not fit it (seams x chunks x overlap^2;
+ * only overlaps above 16 with few seams) take the one-pass form that needs no
+ * partial sums.
+ *
+ * Set-up and memory: CUDA loads a library's device code lazily by default, so
+ * the first call on each device loads this entry point's kernels and, with
+ * them, the 1 MiB array (about 1 MiB plus code).  Make that first call before
+ * handing the device's memory to a pool, or it may fail with TDM_ECUDA; later
+ * calls take no device memory.  Each call outside stream capture looks up the
+ * array's device address (cudaGetSymbolAddress) on the current device, so a
+ * device reset or another current context is followed.  A call under stream
+ * capture uses the address that the last uncaptured call on that device found,
+ * and returns TDM_EUNSUPPORTED when there was none: make the first call, and
+ * one after any cudaDeviceReset, outside capture.
  *
  * All calls on a device share that array and it keeps the last call's partial
  * sums; each call writes every partial sum it reads before reading it, so no
@@ -362,11 +385,9 @@ tdm_status tdm_nonoverlap_drift(tdm_ctx *ctx, const float *maps, const float *re
  * serialised by the caller.
  *
  * Errors: TDM_EINVAL (NULL or misaligned pointers, T < 2, B < 1, overlap
- * outside [1, 32], bad shard fields), TDM_EUNSUPPORTED when the partial sums
- * would exceed TDM_NOALLOC_SCRATCH_FLOATS (seams x chunks x overlap^2; never
- * for overlaps up to 16) or the device index is 64 or more, TDM_ECUDA on a
- * failed launch or symbol lookup.  There is no context to hold an error
- * message. */
+ * outside [1, 32], bad shard fields), TDM_EUNSUPPORTED for a first use under
+ * stream capture (above), TDM_ECUDA on a failed launch or symbol lookup.
+ * There is no context to hold an error message. */
 #define TDM_NOALLOC_SCRATCH_FLOATS 262144
 tdm_status tdm_seam_discrepancy_noalloc(const float *maps, const tdm_tiling *tiling, float *out,
                                         tdm_stream stream);

@@ -71,6 +71,7 @@ _SIGS = {
     "tdm_scan_nonfinite": (_i32, [_vp, _vp, _i64, _vp]),
     "tdm_fma_rate": (_i32, [_vp, ctypes.POINTER(_f64), _vp]),
     "tdm_mds_reconstruct": (_i32, [_vp, _vp, _i64, _vp, _vp, _vp, _vp]),
+    "tdm_fused_lane_map": (_i32, [_i32, _i32, _vp, _i64]),
 }
 for _name, (_res, _args) in _SIGS.items():
     try:
@@ -436,11 +437,27 @@ def seam_discrepancy_noalloc(maps, tiling: Tiling, out):
     import torch
     _need(maps, tiling.n_maps * 4096, "maps")
     _need(out, tiling.C * max(tiling.T - 1, 0), "out")
+    if out.device != maps.device:
+        raise ValueError(f"out is on {out.device}, maps on {maps.device}")
     ct = tiling.c()
-    stream = _vp(torch.cuda.current_stream(maps.device.index).cuda_stream)
-    st = _lib.tdm_seam_discrepancy_noalloc(_ptr(maps, "maps"), ctypes.byref(ct), _ptr(out, "out"), stream)
+    # the C side runs on the current device: make it the one that holds maps
+    with torch.cuda.device(maps.device):
+        stream = _vp(torch.cuda.current_stream(maps.device).cuda_stream)
+        st = _lib.tdm_seam_discrepancy_noalloc(_ptr(maps, "maps"), ctypes.byref(ct), _ptr(out, "out"), stream)
     if st != OK:
         raise TdmError(st, "tdm_seam_discrepancy_noalloc")
+    return out
+
+
+def fused_lane_map(T: int, overlap: int = 12):
+    """The quad each lane of the fused run holds, as a numpy uint32 array
+    ``[17 T, 32]`` of q | r << 4 | k << 10 | paired << 31 (host only; see
+    tdm_fused_lane_map)."""
+    import numpy as np
+    out = np.empty((17 * T, 32), dtype=np.uint32)
+    st = _lib.tdm_fused_lane_map(int(T), int(overlap), out.ctypes.data_as(_vp), out.size)
+    if st != OK:
+        raise TdmError(st, f"tdm_fused_lane_map(T={T}, overlap={overlap})")
     return out
 
 

@@ -153,7 +153,6 @@ void tdm_ctx_destroy(tdm_ctx *ctx) {
     if (ctx == nullptr) return;
     {
         DeviceScope ds(ctx->device);
-        for (auto &kv : ctx->plans) cudaFree(kv.second);
         cudaFree(ctx->d_flags);
         cudaFree(ctx->d_scratch);
     }
@@ -400,14 +399,11 @@ tdm_status tdm_ddim_step(tdm_ctx *ctx, const tdm_schedule *sched, int32_t step, 
     if (w != 0.0f && (s = check_maps(ctx, eps_u, "eps_u")) != TDM_OK) return s;
     DeviceScope ds(ctx->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the projection, when due after this step, runs inside the step's kernel
+    const bool project = t.T > 1 && t.sync_every > 0 && (sched->S - step) % t.sync_every == 0;
     cudaError_t e = tdm::launch_ddim_step(sched->d_coef, step, maps, eps_c, w != 0.0f ? eps_u : nullptr, w,
-                                          sched->eta > 0.0, seed, t, st);
-    if (e != cudaSuccess) return cuda_fail(ctx, e, "ddim_step launch");
-    if (t.T > 1 && t.sync_every > 0 && (sched->S - step) % t.sync_every == 0) {
-        e = tdm::launch_seam_project(maps, t, st);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "seam projection launch");
-    }
-    return TDM_OK;
+                                          sched->eta > 0.0, project, seed, t, st);
+    return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "ddim_step launch");
 }
 
 tdm_status tdm_ddim_run(tdm_ctx *ctx, const tdm_schedule *sched, float *maps, const float *x0, float w, float s_c,
@@ -441,28 +437,8 @@ tdm_status tdm_ddim_run_steps(tdm_ctx *ctx, const tdm_schedule *sched, float *ma
     if (t.n_maps() == 0) return TDM_OK;
     if ((s = check_maps(ctx, maps, "maps")) != TDM_OK || (s = check_maps(ctx, x0, "x0")) != TDM_OK) return s;
     DeviceScope ds(ctx->device);
-    const int ov = t.T > 1 ? t.overlap : 0;
-    uint32_t *plan = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(ctx->mu);
-        auto it = ctx->plans.find({t.T, ov});
-        if (it != ctx->plans.end()) {
-            plan = it->second;
-        } else {
-            std::vector<uint32_t> h = tdm::build_run_plan(t.T, ov);
-            if (h.size() != (size_t)tdm::kUpperQuads * t.T)
-                return fail(ctx, TDM_EUNSUPPORTED, "ddim_run: lane plan has wrong size");
-            cudaError_t e = cudaMalloc(&plan, h.size() * sizeof(uint32_t));
-            if (e == cudaSuccess) e = cudaMemcpy(plan, h.data(), h.size() * sizeof(uint32_t), cudaMemcpyHostToDevice);
-            if (e != cudaSuccess) {
-                cudaFree(plan);
-                return cuda_fail(ctx, e, "lane plan upload");
-            }
-            ctx->plans[{t.T, ov}] = plan;
-        }
-    }
     cudaError_t e = tdm::launch_ddim_run(sched->d_coef, sched->S, first_step, n_steps, maps, x0, w, s_c, s_u,
-                                         sched->eta > 0.0, seed, init_noise != 0, t, plan,
+                                         sched->eta > 0.0, seed, init_noise != 0, t,
                                          static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "ddim_run launch");
 }
@@ -501,8 +477,8 @@ tdm_status tdm_kabsch_stitch(tdm_ctx *ctx, const float *coords, const tdm_tiling
     if (residual_out != nullptr && (reinterpret_cast<uintptr_t>(residual_out) & 3u))
         return fail(ctx, TDM_EINVAL, "residual_out is not 4-byte aligned");
     DeviceScope ds(ctx->device);
-    cudaError_t e = tdm::launch_stitch(coords, t, chain_out, t.T > 1 ? residual_out : nullptr, ctx->d_scratch,
-                                       ctx->scratch_floats, static_cast<cudaStream_t>(stream));
+    cudaError_t e = tdm::launch_stitch(coords, t, chain_out, t.T > 1 ? residual_out : nullptr,
+                                       static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TDM_OK : cuda_fail(ctx, e, "stitch launch");
 }
 

@@ -51,8 +51,6 @@ struct tdm_ctx {
     uint32_t *d_flags = nullptr;         // device status word (TDM_FLAG_*)
     float *d_scratch = nullptr;          // partial sums of the seam discrepancy
     size_t scratch_floats = 0;
-    std::map<std::pair<int, int>, uint32_t *> plans;  // (T, overlap) -> fused-run lane plan
-    std::mutex mu;
 };
 
 namespace tdm {
@@ -62,11 +60,11 @@ cudaError_t launch_init_noise(float *maps, const Tiling &t, uint64_t seed, cudaS
 cudaError_t launch_eps_standin(const StepCoef *coef, int step, const float *maps, const float *x0, float s,
                                int tag, uint64_t seed, const Tiling &t, float *eps, cudaStream_t st);
 cudaError_t launch_ddim_step(const StepCoef *coef, int step, float *maps, const float *eps_c,
-                             const float *eps_u, float w, bool has_eta, uint64_t seed, const Tiling &t,
-                             cudaStream_t st);
+                             const float *eps_u, float w, bool has_eta, bool project, uint64_t seed,
+                             const Tiling &t, cudaStream_t st);
 cudaError_t launch_ddim_run(const StepCoef *coef, int S, int first, int n_steps, float *maps, const float *x0,
                             float w, float s_c, float s_u, bool has_eta, uint64_t seed, bool init_noise,
-                            const Tiling &t, const uint32_t *plan, cudaStream_t st);
+                            const Tiling &t, cudaStream_t st);
 cudaError_t launch_seam_project(float *maps, const Tiling &t, cudaStream_t st);
 cudaError_t launch_seam_sums(const float *maps, const Tiling &t, float *partial, int chunks,
                              cudaStream_t st);
@@ -79,13 +77,11 @@ cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigva
 cudaError_t launch_pdist(const float *coords, int64_t n, float *maps, cudaStream_t st);
 cudaError_t launch_refine(const float *maps, int64_t n, float *coords, int iterations, float *stress,
                           cudaStream_t st);
-cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, float *scratch,
-                          size_t scratch_floats, cudaStream_t st);
+cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, cudaStream_t st);
 cudaError_t launch_philox(const uint32_t *ctr, int64_t n, uint64_t seed, uint32_t *out, cudaStream_t st);
 cudaError_t launch_box_muller(const uint32_t *words, int64_t n_pairs, float *z, cudaStream_t st);
 
 // host helpers
-std::vector<uint32_t> build_run_plan(int T, int overlap);
 int seam_chunks(int64_t n_seams, int B);
 int drift_chunks(int64_t tiles, int B);
 cudaError_t launch_scan_nonfinite(const float *buf, int64_t n, uint32_t *flags, cudaStream_t st);

@@ -104,49 +104,100 @@ __global__ void __launch_bounds__(kMapThreads) eps_standin_kernel(
 
 // ---- one DDIM step ------------------------------------------------------------
 
+// The guided eps and the DDIM update of one entry, in one order for every
+// entry (its own map's, or its partner's across a seam).
 template <bool HAS_U, bool HAS_ETA>
+__device__ __forceinline__ float step_entry(const StepCoef &cf, float wc, float w, float x, float ec, float eu,
+                                            float z) {
+    const float e = HAS_U ? fmaf(wc, ec, -w * eu) : ec;
+    const float y = fmaf(cf.a, x, cf.kb * e);
+    return HAS_ETA ? fmaf(cf.ks, z, y) : y;
+}
+
+// One CTA per map.  With PROJ (the step after which the overlap projection of
+// §4.3.2 is due), the CTA of tile k < T-1 also updates the partner entries of
+// tile k+1 over their shared o x o block and writes the mean of the two
+// updated values to both maps; the CTA of tile k > 0 leaves its own block
+// with tile k-1 to that tile's CTA.  So every entry is read and written by one
+// CTA, and the projection costs no pass of its own.
+template <bool HAS_U, bool HAS_ETA, bool PROJ>
 __global__ void __launch_bounds__(kMapThreads) ddim_step_kernel(
     const StepCoef *__restrict__ coef, int step, float *__restrict__ maps, const float *__restrict__ eps_c,
     const float *__restrict__ eps_u, float w, const PhiloxKeys K, Tiling t) {
+    constexpr int kBlockLd = 33;
     __shared__ float zs[HAS_ETA ? kN * kZLd : 1];
+    __shared__ float zn[HAS_ETA && PROJ ? 32 * kBlockLd : 1];    // the partner's ETA field over the block
     const StepCoef cf = coef[step];
     const float wc = 1.0f + w;
     const int64_t n = t.n_maps();
+    const int o = t.overlap, s = kN - o;
     for (int64_t m = blockIdx.x; m < n; m += gridDim.x) {
+        const int64_t tile = m / t.B;
+        const int b = (int)(m - tile * t.B);
+        const int c = (int)(tile / t.T), k = (int)(tile - (int64_t)c * t.T);
+        const bool right = PROJ && k < t.T - 1, left = PROJ && k > 0;
         if (HAS_ETA) {
-            const int64_t tile = m / t.B;
-            const int b = (int)(m - tile * t.B);
-            const int c = (int)(tile / t.T), k = (int)(tile - (int64_t)c * t.T);
             const uint64_t g = noise_id(t.sample_id_base, c, t.T, k, t.B_total, t.b_offset, b);
             fill_symmetric_noise(zs, g, TDM_STREAM_ETA, (uint32_t)step, K);
+            if (PROJ && right) {
+                // upper quads of the partner's o x o block (map id g + B_total), mirrored
+                const uint64_t gn = g + (uint64_t)t.B_total;
+                const int oq4 = (o + 3) >> 2;
+                for (int u = threadIdx.x; u < o * oq4; u += blockDim.x) {
+                    const int r = u / oq4, q = u - r * oq4;
+                    if (4 * q + 3 < r) continue;
+                    const float4 z = quad_normals(r, q, (uint32_t)step, gn, TDM_STREAM_ETA, K);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * q + e;
+                        if (j >= r && j < o) {
+                            zn[r * kBlockLd + j] = comp(z, e);
+                            zn[j * kBlockLd + r] = comp(z, e);
+                        }
+                    }
+                }
+            }
             __syncthreads();
         }
         float *xm = maps + m * kMapFloats;
         const float *ec = eps_c + m * kMapFloats;
         const float *eu = HAS_U ? eps_u + m * kMapFloats : nullptr;
+        float *xn = xm + (int64_t)t.B * kMapFloats;    // the same sample of tile k+1
+        const float *ecn = ec + (int64_t)t.B * kMapFloats;
+        const float *eun = HAS_U ? eu + (int64_t)t.B * kMapFloats : nullptr;
 #pragma unroll 4
         for (int p = threadIdx.x; p < kMapFloats / 4; p += kMapThreads) {
-            float4 x = ld4(xm + 4 * p);
-            float4 e = ldg4(ec + 4 * p);
-            if (HAS_U) {
-                const float4 v = ldg4(eu + 4 * p);
-                e.x = wc * e.x - w * v.x;
-                e.y = wc * e.y - w * v.y;
-                e.z = wc * e.z - w * v.z;
-                e.w = wc * e.w - w * v.w;
+            const int r = p >> 4, c0 = 4 * (p & 15);
+            const float4 x = ld4(xm + 4 * p);
+            const float4 e = ldg4(ec + 4 * p);
+            const float4 v = HAS_U ? ldg4(eu + 4 * p) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float *z = HAS_ETA ? zs + r * kZLd + c0 : nullptr;
+            float4 y;
+            y.x = step_entry<HAS_U, HAS_ETA>(cf, wc, w, x.x, e.x, v.x, HAS_ETA ? z[0] : 0.f);
+            y.y = step_entry<HAS_U, HAS_ETA>(cf, wc, w, x.y, e.y, v.y, HAS_ETA ? z[1] : 0.f);
+            y.z = step_entry<HAS_U, HAS_ETA>(cf, wc, w, x.z, e.z, v.z, HAS_ETA ? z[2] : 0.f);
+            y.w = step_entry<HAS_U, HAS_ETA>(cf, wc, w, x.w, e.w, v.w, HAS_ETA ? z[3] : 0.f);
+            const bool in_left = left && r < o && c0 < o;
+            const bool in_right = right && r >= s && c0 + 3 >= s;
+            if (!(PROJ && (in_left || in_right))) {
+                st4(xm + 4 * p, y);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int col = c0 + u;
+                    if (in_left && col < o) continue;              // written by tile k-1's CTA
+                    float val = comp(y, u);
+                    if (in_right && col >= s) {
+                        const int off = (r - s) * kN + (col - s);
+                        const float yn = step_entry<HAS_U, HAS_ETA>(
+                            cf, wc, w, xn[off], __ldg(ecn + off), HAS_U ? __ldg(eun + off) : 0.f,
+                            HAS_ETA ? zn[(r - s) * kBlockLd + (col - s)] : 0.f);
+                        val = 0.5f * (val + yn);
+                        xn[off] = val;
+                    }
+                    xm[4 * p + u] = val;
+                }
             }
-            x.x = fmaf(cf.a, x.x, cf.kb * e.x);
-            x.y = fmaf(cf.a, x.y, cf.kb * e.y);
-            x.z = fmaf(cf.a, x.z, cf.kb * e.z);
-            x.w = fmaf(cf.a, x.w, cf.kb * e.w);
-            if (HAS_ETA) {
-                const float *z = zs + (p >> 4) * kZLd + 4 * (p & 15);
-                x.x = fmaf(cf.ks, z[0], x.x);
-                x.y = fmaf(cf.ks, z[1], x.y);
-                x.z = fmaf(cf.ks, z[2], x.z);
-                x.w = fmaf(cf.ks, z[3], x.w);
-            }
-            st4(xm + 4 * p, x);
         }
         if (HAS_ETA) __syncthreads();
     }
@@ -162,14 +213,110 @@ __global__ void __launch_bounds__(kMapThreads) ddim_step_kernel(
 // of such a pair in lanes l and l^16 of one warp, so the projection is one
 // register exchange; no CTA ever waits on another.
 
+// The lanes of one chain-sample (17 T warps) cover the 544 T upper row
+// quads of its T tiles.  With overlap o = 4 oq and stride s = 64 - o, the
+// upper quads of the o x o overlap block of a seam are indexed u in row-major
+// order (row i < o, column quad jq < oq, 4 jq + 3 >= i: Q = 2 oq (oq + 1) of
+// them), and pair p = k Q + u joins quad (s + i, sq + jq) of tile k with quad
+// (i, jq) of tile k + 1 (sq = s / 4).  Warp w < P / 16 holds pairs 16 w ..
+// 16 w + 15, first quads in lanes 0-15 and second quads in lanes l + 16; the
+// next warp holds the last P % 16 pairs in the same way and fills its other
+// lanes two at a time (l, l + 16) with the first singles; the remaining warps
+// hold 32 singles each.  The singles are every other upper quad in the order
+// tile, row, column quad.
+//
+// Two constant tables, built at compile time, hold what depends only on oq:
+// the (i, jq) of each block quad u, and for each kind of tile (with or without
+// a left block, with or without a right block) the (r, q) of its singles in
+// order.  A lane's descriptor is then two divisions and one table read.
+struct LaneTables {
+    uint16_t single[9][4][kUpperQuads];    // [oq][left | right << 1][index] -> r << 4 | q
+    uint8_t pair[9][144];                  // [oq][u] -> i | jq << 5
+};
+
+constexpr LaneTables make_lane_tables() {
+    LaneTables t{};
+    for (int oq = 0; oq <= 8; ++oq) {
+        const int ov = 4 * oq, s = kN - ov, sq = kQuadsPerRow - oq;
+        int u = 0;
+        for (int i = 0; i < ov; ++i)
+            for (int jq = 0; jq < oq; ++jq)
+                if (4 * jq + 3 >= i) t.pair[oq][u++] = (uint8_t)(i | jq << 5);
+        for (int kind = 0; kind < 4; ++kind) {
+            const bool L = (kind & 1) != 0, R = (kind & 2) != 0;
+            int n = 0;
+            for (int r = 0; r < kN; ++r)
+                for (int q = 0; q < kQuadsPerRow; ++q) {
+                    if (4 * q + 3 < r) continue;
+                    const bool left = L && r < ov && q < oq, right = R && r >= s && q >= sq;
+                    if (!left && !right) t.single[oq][kind][n++] = (uint16_t)(r << 4 | q);
+                }
+        }
+    }
+    return t;
+}
+
+__device__ const LaneTables kLaneTablesDev = make_lane_tables();
+
+// x / d for 0 <= x < 2^31 and 0 < d < 2^16, with m = ceil(2^32 / d): the
+// product's top word is x / d or one more, and one comparison corrects it.
+__host__ __device__ inline int div_magic(int x, int d, uint32_t m) {
+    int k = (int)(((uint64_t)(uint32_t)x * m) >> 32);
+    if (k * d > x) --k;
+    return k;
+}
+
+__host__ __device__ inline uint32_t div_magic_of(int d) {
+    return d > 1 ? (uint32_t)((0x100000000ULL + (uint64_t)d - 1) / (uint64_t)d) : 0xFFFFFFFFu;
+}
+
+// q | r << 4 | k << 10 | paired << 31 of lane `lane` of warp `wi`; mq and
+// mmid are div_magic_of(Q) and div_magic_of(544 - 2 Q).
+__host__ __device__ inline uint32_t run_lane_desc(const LaneTables &tab, int T, int overlap, int wi, int lane,
+                                                  uint32_t mq, uint32_t mmid) {
+    const int oq = overlap >> 2, sq = kQuadsPerRow - oq;
+    const int Q = 2 * oq * (oq + 1);
+    const int P = (T - 1) * Q, Pw = P >> 4, Pr = P & 15;
+    const int pl = lane & 15;
+    const bool hi = lane >= 16;
+    if (wi < Pw || (wi == Pw && pl < Pr)) {
+        const int p = 16 * wi + pl;
+        const int k = div_magic(p, Q, mq);
+        const int e = tab.pair[oq][p - k * Q];
+        const int i = e & 31, jq = e >> 5;
+        return hi ? ((uint32_t)jq | (uint32_t)i << 4 | (uint32_t)(k + 1) << 10 | 0x80000000u)
+                  : ((uint32_t)(sq + jq) | (uint32_t)(4 * sq + i) << 4 | (uint32_t)k << 10 | 0x80000000u);
+    }
+    int si;
+    if (wi == Pw && Pr > 0)
+        si = 2 * (pl - Pr) + (hi ? 1 : 0);
+    else
+        si = (Pr > 0 ? 2 * (16 - Pr) : 0) + 32 * (wi - Pw - (Pr > 0 ? 1 : 0)) + lane;
+    // the tile: tile 0 and tile T-1 lose one block each, the others two
+    const int n_first = kUpperQuads - (T > 1 ? Q : 0), n_mid = kUpperQuads - 2 * Q;
+    int k = 0, sl = si;
+    if (si >= n_first) {
+        const int rem = si - n_first;
+        k = 1 + div_magic(rem, n_mid, mmid);
+        sl = rem - (k - 1) * n_mid;
+        if (k >= T - 1) {
+            k = T - 1;
+            sl = rem - (T - 2) * n_mid;
+        }
+    }
+    const int kind = (k > 0 ? 1 : 0) | (k < T - 1 ? 2 : 0);
+    const uint32_t rq = tab.single[oq][kind][sl];
+    return (rq & 15u) | (rq >> 4) << 4 | (uint32_t)k << 10;
+}
+
 struct RunArgs {
     const StepCoef *coef;
     float *maps;
     const float *x0;
-    const uint32_t *plan;      // [17 T][32] lane descriptors
     int64_t total_warps;       // C * B * 17 T
     int64_t B_total, b_off, base;
-    int S, T, B, sync_every, warps_per_chain;
+    int S, T, B, overlap, sync_every, warps_per_chain;
+    uint32_t mq, mmid;         // division constants of the lane descriptors
     int first, last;           // steps first, first-1, .., last (first = S-1, last = 0 for a whole run)
     float cc, cu;              // (1 + w) s_c and w s_u
     PhiloxKeys K;
@@ -248,7 +395,7 @@ __global__ void __launch_bounds__(256) ddim_run_kernel(const RunArgs a) {
     if (gw >= a.total_warps) return;
     const int64_t cs = gw / a.warps_per_chain;               // chain-sample c * B + b
     const int wi = (int)(gw - cs * a.warps_per_chain);
-    const uint32_t d = __ldg(a.plan + wi * 32 + lane);
+    const uint32_t d = run_lane_desc(kLaneTablesDev, a.T, a.overlap, wi, lane, a.mq, a.mmid);
     const int q = d & 15, r = (d >> 4) & 63, k = (d >> 10) & 0xFFFF;
     const bool paired = (d >> 31) != 0;
     const int c = (int)(cs / a.B), b = (int)(cs - (int64_t)c * a.B);
@@ -374,43 +521,22 @@ int grid_for(int64_t work_items, int per_sm) {
 
 // ---- host side -------------------------------------------------------------------
 
-std::vector<uint32_t> build_run_plan(int T, int overlap) {
-    const int s = kN - overlap, sq = s / 4, oq = overlap / 4;
-    auto desc = [](int k, int r, int q, bool paired) {
-        return (uint32_t)q | ((uint32_t)r << 4) | ((uint32_t)k << 10) | (paired ? 0x80000000u : 0u);
-    };
-    std::vector<std::pair<uint32_t, uint32_t>> pairs;
-    std::vector<uint32_t> singles;
-    for (int k = 0; k < T; ++k)
-        for (int r = 0; r < kN; ++r)
-            for (int q = 0; q < kQuadsPerRow; ++q) {
-                if (4 * q + 3 < r) continue;                       // not in the folded state
-                const bool right = k < T - 1 && r >= s && q >= sq;
-                const bool left = k > 0 && r < overlap && q < oq;
-                if (right)
-                    pairs.emplace_back(desc(k, r, q, true), desc(k + 1, r - s, q - sq, true));
-                else if (!left)
-                    singles.push_back(desc(k, r, q, false));
-            }
-    std::vector<uint32_t> plan;
-    plan.reserve((size_t)kUpperQuads * T);
-    size_t si = 0;
-    for (size_t p0 = 0; p0 < pairs.size(); p0 += 16) {
-        uint32_t wl[32];
-        for (int l = 0; l < 16; ++l) {
-            if (p0 + l < pairs.size()) {
-                wl[l] = pairs[p0 + l].first;
-                wl[l + 16] = pairs[p0 + l].second;
-            } else {
-                wl[l] = singles[si++];
-                wl[l + 16] = singles[si++];
-            }
-        }
-        plan.insert(plan.end(), wl, wl + 32);
-    }
-    plan.insert(plan.end(), singles.begin() + si, singles.end());
-    return plan;
+}  // namespace tdm
+
+extern "C" tdm_status tdm_fused_lane_map(int32_t T, int32_t overlap, uint32_t *out, int64_t n) {
+    if (T < 1 || T > 0xFFFF || out == nullptr) return TDM_EINVAL;
+    const int ov = T > 1 ? overlap : 0;
+    if (ov < 0 || ov > 32 || ov % 4 != 0 || (T > 1 && ov < 4)) return TDM_EINVAL;
+    if (n < (int64_t)tdm::kUpperQuads * T) return TDM_EINVAL;
+    static const tdm::LaneTables tab = tdm::make_lane_tables();
+    const int oq = ov >> 2, Q = 2 * oq * (oq + 1);
+    const uint32_t mq = tdm::div_magic_of(Q), mmid = tdm::div_magic_of(tdm::kUpperQuads - 2 * Q);
+    for (int wi = 0; wi < 17 * T; ++wi)
+        for (int l = 0; l < 32; ++l) out[(int64_t)wi * 32 + l] = tdm::run_lane_desc(tab, T, ov, wi, l, mq, mmid);
+    return TDM_OK;
 }
+
+namespace tdm {
 
 cudaError_t launch_init_noise(float *maps, const Tiling &t, uint64_t seed, cudaStream_t st) {
     const int64_t items = t.n_maps() * kUpperQuads;
@@ -428,19 +554,25 @@ cudaError_t launch_eps_standin(const StepCoef *coef, int step, const float *maps
 }
 
 cudaError_t launch_ddim_step(const StepCoef *coef, int step, float *maps, const float *eps_c,
-                             const float *eps_u, float w, bool has_eta, uint64_t seed, const Tiling &t,
-                             cudaStream_t st) {
+                             const float *eps_u, float w, bool has_eta, bool project, uint64_t seed,
+                             const Tiling &t, cudaStream_t st) {
     const int grid = grid_for(t.n_maps(), 8);
     const PhiloxKeys K = philox_keys(seed);
     const bool has_u = eps_u != nullptr && w != 0.0f;
-    if (has_u && has_eta)
-        ddim_step_kernel<true, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, K, t);
-    else if (has_u)
-        ddim_step_kernel<true, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, eps_u, w, K, t);
-    else if (has_eta)
-        ddim_step_kernel<false, true><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, K, t);
-    else
-        ddim_step_kernel<false, false><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, nullptr, w, K, t);
+    const int v = (has_u ? 4 : 0) | (has_eta ? 2 : 0) | (project && t.T > 1 ? 1 : 0);
+#define TDM_STEP(U, E, P)                                                                                    \
+    ddim_step_kernel<U, E, P><<<grid, kMapThreads, 0, st>>>(coef, step, maps, eps_c, U ? eps_u : nullptr, w, K, t)
+    switch (v) {
+        case 7: TDM_STEP(true, true, true); break;
+        case 6: TDM_STEP(true, true, false); break;
+        case 5: TDM_STEP(true, false, true); break;
+        case 4: TDM_STEP(true, false, false); break;
+        case 3: TDM_STEP(false, true, true); break;
+        case 2: TDM_STEP(false, true, false); break;
+        case 1: TDM_STEP(false, false, true); break;
+        default: TDM_STEP(false, false, false); break;
+    }
+#undef TDM_STEP
     return cudaGetLastError();
 }
 
@@ -464,14 +596,19 @@ static cudaError_t run_variant(const RunArgs &a, int grid, int threads, size_t s
 
 cudaError_t launch_ddim_run(const StepCoef *coef, int S, int first, int n_steps, float *maps, const float *x0,
                             float w, float s_c, float s_u, bool has_eta, uint64_t seed, bool init_noise,
-                            const Tiling &t, const uint32_t *plan, cudaStream_t st) {
+                            const Tiling &t, cudaStream_t st) {
     RunArgs a;
     a.first = first;
     a.last = first - n_steps + 1;
     a.coef = coef;
     a.maps = maps;
     a.x0 = x0;
-    a.plan = plan;
+    a.overlap = t.T > 1 ? t.overlap : 0;
+    {
+        const int oq = a.overlap >> 2, Q = 2 * oq * (oq + 1);
+        a.mq = div_magic_of(Q);
+        a.mmid = div_magic_of(kUpperQuads - 2 * Q);
+    }
     a.warps_per_chain = 17 * t.T;
     a.total_warps = (int64_t)t.C * t.B * a.warps_per_chain;
     a.B_total = t.B_total;
