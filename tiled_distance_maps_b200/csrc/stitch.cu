@@ -9,12 +9,12 @@
 // maps compose along the chain into tile 0's frame; overlap beads take the
 // mean of their two aligned copies.
 //
-// Chains of up to kFusedMaxT tiles take one pass: a CTA per (chain, sample)
-// pair, whose first warp aligns the seams and composes the maps by a shuffle
-// scan, 32 tiles at a time, into shared memory, after which all its threads
-// place the pair's beads.  Longer chains take two passes over chunks of pairs
-// whose maps fit the context scratch: the same alignment into global memory,
-// then one thread per group of chain beads.
+// One CTA per (chain, sample) pair walks the chain in chunks of 32 tiles.  It
+// stages the chunk's tiles (and the next one) in shared memory, once; its first
+// warp aligns the chunk's seams, a lane per seam, and composes the maps by a
+// shuffle scan, carried from chunk to chunk; then all its threads place the
+// chunk's beads from the staged tiles.  Each tile is read from memory once,
+// and chains of any length take this one pass.
 #include "common.cuh"
 
 namespace tdm {
@@ -264,65 +264,12 @@ __device__ __forceinline__ Rigid chunk_maps(const float *P, const float *Q, int 
     return gk;
 }
 
-// 4-byte asynchronous global -> shared copy (the copies of a chunk are all in
-// flight before the warp waits for them)
+// 4-byte asynchronous global -> shared copy (a chunk's copies are all in
+// flight before the CTA waits for them)
 __device__ __forceinline__ void async_copy4(float *dst, const float *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                  "l"(src)
                  : "memory");
-}
-
-// The maps of every tile of pair (c, b) into out[0 .. T) and its residuals
-// into resid (warp-wide): the seam beads of 32 tiles at a time are staged in
-// shared memory (sbeads: [2][32][3o+1], P then Q per lane) by coalesced
-// warp-wide asynchronous copies (per-lane stride 3o+1 floats, odd, so the
-// lanes' reads do not conflict); out may be global or shared memory.
-__device__ __forceinline__ void pair_maps(const float *__restrict__ coords, int T, int B, int o, int c, int b,
-                                          int64_t pair, float *sbeads, float *__restrict__ resid, Rigid *out) {
-    const int lane = threadIdx.x & 31;
-    const int s = kN - o;
-    const int n3 = 3 * o, ld = 3 * o + 1;
-    float *sP = sbeads, *sQ = sbeads + 32 * ld;
-    Rigid carry = identity(), carry_prev = identity();
-    for (int k0 = 0; k0 < T; k0 += 32) {
-        const int nseam = min(32, T - 1 - k0);    // seams k0 .. k0+nseam-1
-        __syncwarp();
-        for (int r = 0; r < nseam; ++r) {
-            const float *Pg = coords + (((int64_t)c * T + k0 + r) * B + b) * (kN * 3) + s * 3;
-            const float *Qg = coords + (((int64_t)c * T + k0 + r + 1) * B + b) * (kN * 3);
-            for (int i = lane; i < n3; i += 32) {
-                async_copy4(sP + r * ld + i, Pg + i);
-                async_copy4(sQ + r * ld + i, Qg + i);
-            }
-        }
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
-        __syncwarp();
-        const Rigid gk = chunk_maps(sP + lane * ld, sQ + lane * ld, T, o, k0, pair, resid, carry, carry_prev);
-        if (k0 + lane < T) out[k0 + lane] = gk;
-    }
-}
-
-// Pass 1 of the two-pass form: one warp (one CTA) per (chain, sample) of
-// pairs [pair0, pair0 + n): every tile's map into gmaps[(pair - pair0) * T + k]
-// and the residuals into resid.
-__global__ void __launch_bounds__(32) stitch_align_kernel(const float *__restrict__ coords, int T, int B, int o,
-                                                          int64_t pair0, Rigid *__restrict__ gmaps,
-                                                          float *__restrict__ resid) {
-    extern __shared__ float sbeads[];    // [2][32][3o+1]
-    const int64_t q = blockIdx.x;
-    const int64_t pair = pair0 + q;
-    const int c = (int)(pair / B), b = (int)(pair - (int64_t)(pair / B) * B);
-    pair_maps(coords, T, B, o, c, b, pair, sbeads, resid, gmaps + q * T);
-}
-
-__device__ __forceinline__ Rigid load_map(const Rigid *g) {
-    const float4 *v = reinterpret_cast<const float4 *>(g);
-    const float4 a = __ldg(v), b = __ldg(v + 1), c = __ldg(v + 2);
-    Rigid o;
-    o.r[0] = a.x, o.r[1] = a.y, o.r[2] = a.z, o.r[3] = a.w;
-    o.r[4] = b.x, o.r[5] = b.y, o.r[6] = b.z, o.r[7] = b.w;
-    o.r[8] = c.x, o.t[0] = c.y, o.t[1] = c.z, o.t[2] = c.w;
-    return o;
 }
 
 __device__ __forceinline__ Rigid smem_map(const Rigid *g) {
@@ -335,106 +282,88 @@ __device__ __forceinline__ Rigid smem_map(const Rigid *g) {
     return o;
 }
 
-// Chain beads [p, p + G) of pair (c, b) from its tiles' coordinates and maps
-// (maps: the pair's T maps, global when GLOBAL_MAPS, else shared).  Tile k owns
-// chain positions [k s, k s + s), the last tile [k s, k s + 64); the first o
-// beads of tile k > 0 are the mean of tile k-1's and tile k's aligned copies.
-// G = 4 needs o % 4 == 0: four beads then stay in one tile and on one side of
-// the overlap boundary, and their 12 coordinates are 16-byte aligned in the
-// tile and in the chain.
-template <int G, bool GLOBAL_MAPS>
-__device__ __forceinline__ void place_group(const float *__restrict__ coords, int T, int B, int o, int c, int b,
-                                            int p, const Rigid *maps, float *dst) {
-    const int s = kN - o;
-    int k = p / s;
-    if (k > T - 1) k = T - 1;
-    const int j = p - k * s;
-    // both rounds of loads (the tile's beads and map; for overlap beads also
-    // the previous tile's) are issued before any arithmetic
-    const bool ov = k > 0 && j < o;
-    float x[3 * G], xp[3 * G], y[3 * G];
-    const float *xk = coords + (((int64_t)c * T + k) * B + b) * (kN * 3) + 3 * j;
-    const float *xq = coords + (((int64_t)c * T + (ov ? k - 1 : k)) * B + b) * (kN * 3) + 3 * (s + j);
-    const Rigid gk = GLOBAL_MAPS ? load_map(maps + k) : smem_map(maps + k);
-    Rigid gp = gk;
-    if constexpr (G == 4) {
-#pragma unroll
-        for (int v = 0; v < 3; ++v) *reinterpret_cast<float4 *>(x + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xk) + v);
-        if (ov) {
-#pragma unroll
-            for (int v = 0; v < 3; ++v)
-                *reinterpret_cast<float4 *>(xp + 4 * v) = __ldg(reinterpret_cast<const float4 *>(xq) + v);
-            gp = GLOBAL_MAPS ? load_map(maps + k - 1) : smem_map(maps + k - 1);
-        }
-    } else {
-#pragma unroll
-        for (int v = 0; v < 3 * G; ++v) x[v] = __ldg(xk + v);
-        if (ov) {
-#pragma unroll
-            for (int v = 0; v < 3 * G; ++v) xp[v] = __ldg(xq + v);
-            gp = GLOBAL_MAPS ? load_map(maps + k - 1) : smem_map(maps + k - 1);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < G; ++u) apply(gk, x + 3 * u, y + 3 * u);
-    if (ov) {
-#pragma unroll
-        for (int u = 0; u < G; ++u) {
-            float y1[3];
-            apply(gp, xp + 3 * u, y1);
-#pragma unroll
-            for (int d = 0; d < 3; ++d) y[3 * u + d] = 0.5f * (y1[d] + y[3 * u + d]);
-        }
-    }
-    if constexpr (G == 4) {
-#pragma unroll
-        for (int v = 0; v < 3; ++v) reinterpret_cast<float4 *>(dst)[v] = *reinterpret_cast<const float4 *>(y + 4 * v);
-    } else {
-#pragma unroll
-        for (int v = 0; v < 3 * G; ++v) dst[v] = y[v];
-    }
+__device__ __forceinline__ void smem_store_map(Rigid *g, const Rigid &m) {
+    float4 *v = reinterpret_cast<float4 *>(g);
+    v[0] = make_float4(m.r[0], m.r[1], m.r[2], m.r[3]);
+    v[1] = make_float4(m.r[4], m.r[5], m.r[6], m.r[7]);
+    v[2] = make_float4(m.r[8], m.t[0], m.t[1], m.t[2]);
 }
 
-// Pass 2 of the two-pass form: one thread per G beads of the chains of pairs
-// [pair0, pair0 + n).  32-bit indices: a chunk holds n L <= (scratch / 12T) *
-// 64T beads, and pairs < 2^31 is checked by the caller.
-template <int G>
-__global__ void __launch_bounds__(256) stitch_place_kernel(const float *__restrict__ coords, int T, int B, int o,
-                                                           int pair0, int n, const Rigid *__restrict__ gmaps,
-                                                           float *__restrict__ chain) {
-    const int s = kN - o;
-    const int L = kN + (T - 1) * s;
-    const int LG = L / G;
-    const int total = n * LG;
-    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
-        const int q = idx / LG;
-        const int p = (idx - q * LG) * G;
-        const int pair = pair0 + q;
-        const int c = pair / B, b = pair - (pair / B) * B;
-        place_group<G, true>(coords, T, B, o, c, b, p, gmaps + (int64_t)q * T, chain + ((int64_t)pair * L + p) * 3);
-    }
-}
+constexpr int kStitchThreads = 128;
+constexpr int kChunk = 32;                 // seams aligned per chunk, a lane each
+constexpr int kSlots = kChunk + 1;         // tiles staged per chunk: its 32 and the next
+constexpr int kTileLd = kN * 3 + 1;        // 193 floats: odd, so the lanes' reads of their seams do not conflict
+// shared memory: the maps of the chunk's tiles and of the tile before it, the
+// staged tiles, and the last o beads of the tile before the chunk
+constexpr int kMapsFloats = (kSlots + 1) * 12;
+constexpr int kStitchSmemFloats = kMapsFloats + kSlots * kTileLd + 96;
 
-// The one-pass form for chains of at most kFusedMaxT tiles: one CTA of 128
-// threads per (chain, sample) pair, 7 CTAs per SM (72 registers, no spills),
-// so that 1036 pairs are resident at once.  Warp 0 computes the pair's maps into
-// shared memory (pair_maps), then all threads place its beads.
-constexpr int kFusedMaxT = 512;
-constexpr int kFusedThreads = 128;
-
-template <int G>
-__global__ void __launch_bounds__(kFusedThreads, 7) stitch_kernel(const float *__restrict__ coords, int T, int B, int o,
-                                                     float *__restrict__ chain, float *__restrict__ resid) {
-    extern __shared__ __align__(16) float sm[];    // [2][32][3o+1] bead staging, then [T] maps
-    Rigid *smaps = reinterpret_cast<Rigid *>(sm + 2 * 32 * (3 * o + 1));
+// One CTA per (chain, sample) pair.  Tile k owns chain positions [k s, k s + s),
+// the last tile [k s, k s + 64); the first o beads of tile k > 0 are the mean of
+// tile k-1's and tile k's aligned copies.  Bit for bit the arithmetic of the
+// alignment (align_seam), the scan (chunk_maps) and the placement (apply, then
+// the mean) does not depend on the chunking.
+__global__ void __launch_bounds__(kStitchThreads, 7) stitch_kernel(const float *__restrict__ coords, int T, int B,
+                                                                   int o, float *__restrict__ chain,
+                                                                   float *__restrict__ resid) {
+    extern __shared__ __align__(16) float sm[];
+    Rigid *smaps = reinterpret_cast<Rigid *>(sm);           // [0, 32]: tiles k0 .. k0+31; [32]: tile k0-1
+    float *stile = sm + kMapsFloats;                         // [33][193]: tiles k0 .. k0+32
+    float *sprev = stile + kSlots * kTileLd;                 // tile k0-1's beads s .. 63
     const int64_t pair = blockIdx.x;
     const int c = (int)(pair / B), b = (int)(pair - (int64_t)(pair / B) * B);
-    if (threadIdx.x < 32) pair_maps(coords, T, B, o, c, b, pair, sm, resid, smaps);
-    __syncthreads();
-    const int L = kN + (T - 1) * (kN - o);
+    const int s = kN - o;
+    const int L = kN + (T - 1) * s;
+    const int tid = threadIdx.x;
     float *dst = chain + pair * (int64_t)L * 3;
-    for (int g = threadIdx.x; g < L / G; g += blockDim.x)
-        place_group<G, false>(coords, T, B, o, c, b, g * G, smaps, dst + (int64_t)g * G * 3);
+    Rigid carry = identity(), carry_prev = identity();       // warp 0: G_{k0}, G_{k0-1}
+    for (int k0 = 0; k0 < T; k0 += kChunk) {
+        const int nt = min(kSlots, T - k0);                  // tiles staged
+        const int nc = min(kChunk, T - k0);                  // tiles placed
+        for (int i = 0; i < nt; ++i) {
+            const float *src = coords + (((int64_t)c * T + k0 + i) * B + b) * (kN * 3);
+            for (int e = tid; e < kN * 3; e += kStitchThreads) async_copy4(stile + i * kTileLd + e, src + e);
+        }
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+        __syncthreads();
+        if (tid < 32) {
+            const int lane = tid;
+            if (lane == 0) smem_store_map(smaps + kChunk, carry_prev);
+            const Rigid gk = chunk_maps(stile + lane * kTileLd + 3 * s, stile + (lane + 1) * kTileLd, T, o, k0, pair,
+                                        resid, carry, carry_prev);
+            if (lane < nc) smem_store_map(smaps + lane, gk);
+        }
+        __syncthreads();
+        // the chunk's beads: nc * s of them, plus the last tile's o beyond its stride
+        const int nb = nc * s + (k0 + nc == T ? o : 0);
+        for (int idx = tid; idx < nb; idx += kStitchThreads) {
+            int kl = idx / s;
+            if (kl > nc - 1) kl = nc - 1;
+            const int j = idx - kl * s;
+            const int k = k0 + kl;
+            float x[3], y[3];
+#pragma unroll
+            for (int d = 0; d < 3; ++d) x[d] = stile[kl * kTileLd + 3 * j + d];
+            apply(smem_map(smaps + kl), x, y);
+            if (k > 0 && j < o) {
+                float xp[3], y1[3];
+                const float *bp = kl > 0 ? stile + (kl - 1) * kTileLd + 3 * (s + j) : sprev + 3 * j;
+#pragma unroll
+                for (int d = 0; d < 3; ++d) xp[d] = bp[d];
+                apply(smem_map(smaps + (kl > 0 ? kl - 1 : kChunk)), xp, y1);
+#pragma unroll
+                for (int d = 0; d < 3; ++d) y[d] = 0.5f * (y1[d] + y[d]);
+            }
+            float *out = dst + ((int64_t)k * s + j) * 3;
+#pragma unroll
+            for (int d = 0; d < 3; ++d) out[d] = y[d];
+        }
+        __syncthreads();
+        // the chunk's last tile is the next chunk's tile before it
+        if (k0 + kChunk < T)
+            for (int e = tid; e < 3 * o; e += kStitchThreads) sprev[e] = stile[(kChunk - 1) * kTileLd + 3 * s + e];
+        __syncthreads();
+    }
 }
 
 }  // namespace
@@ -442,42 +371,15 @@ __global__ void __launch_bounds__(kFusedThreads, 7) stitch_kernel(const float *_
 
 namespace tdm {
 
-cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, float *scratch,
-                          size_t scratch_floats, cudaStream_t st) {
+cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, float *resid, cudaStream_t st) {
     const int64_t pairs = (int64_t)t.C * t.B;
     if (pairs <= 0) return cudaSuccess;
     if (pairs > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const int o = t.T > 1 ? t.overlap : 0;
-    const int64_t per_pair = (int64_t)t.T * (int64_t)(sizeof(Rigid) / sizeof(float));
-    // T <= 65535 (checked with the tiling) keeps one pair's maps within the scratch
-    const int64_t chunk = scratch == nullptr ? 0 : (int64_t)scratch_floats / per_pair;
-    if (chunk < 1) return cudaErrorInvalidValue;
-    const bool vec = o % 4 == 0;
-    if (t.T <= kFusedMaxT) {
-        // 2 * 32 * (3o + 1) floats: a multiple of 16 bytes, so the maps that follow are aligned
-        const size_t smem = sizeof(float) * 2 * 32 * (3 * o + 1) + sizeof(Rigid) * (size_t)t.T;
-        if (vec)
-            stitch_kernel<4><<<(unsigned)pairs, kFusedThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
-        else
-            stitch_kernel<1><<<(unsigned)pairs, kFusedThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
-        return cudaGetLastError();
-    }
-    Rigid *gmaps = reinterpret_cast<Rigid *>(scratch);
-    for (int64_t p0 = 0; p0 < pairs; p0 += chunk) {
-        const int64_t n = pairs - p0 < chunk ? pairs - p0 : chunk;
-        const size_t smem = sizeof(float) * 2 * 32 * (3 * o + 1);
-        stitch_align_kernel<<<(unsigned)n, 32, smem, st>>>(coords, t.T, t.B, o, p0, gmaps, resid);
-        const int64_t beads = n * (kN + (int64_t)(t.T - 1) * (kN - o));
-        int64_t blocks = ((vec ? beads / 4 : beads) + 255) / 256;
-        if (blocks > 148LL * 64) blocks = 148LL * 64;
-        if (vec)
-            stitch_place_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(coords, t.T, t.B, o, (int)p0, (int)n, gmaps, chain);
-        else
-            stitch_place_kernel<1><<<(unsigned)blocks, 256, 0, st>>>(coords, t.T, t.B, o, (int)p0, (int)n, gmaps, chain);
-        const cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    const size_t smem = sizeof(float) * kStitchSmemFloats;
+    static_assert(kMapsFloats % 4 == 0, "16-byte alignment of the staged maps");
+    stitch_kernel<<<(unsigned)pairs, kStitchThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
+    return cudaGetLastError();
 }
 
 }  // namespace tdm
