@@ -8,14 +8,15 @@
 // Per map, one warp stages D in shared memory by 16-byte asynchronous copies
 // (the warp's next map is brought into L2 by one bulk prefetch issued when the
 // current map's eigen-solve is done, so those copies wait on L2 rather than
-// DRAM) and forms B.  The top
+// DRAM) and forms B = -1/8 J E J from E = (D + D^T)^2 entrywise.  The top
 // eigenpairs come from subspace iteration on three vectors with a
 // Rayleigh-Ritz step (a 3 x 3 Jacobi eigen-solve) every iteration, stopping
 // when the residual of the three Ritz pairs is below kTol * |l_1|.  The start
 // basis is the three columns of B with the largest diagonal entries (the
 // points farthest from the centroid): for an exact Euclidean map they already
 // span the answer.  Row l of B stays in registers for the products; row l+32
-// is read from shared memory.
+// is read from shared memory.  Forming B and the products run in packed
+// float32 (two columns per instruction), which halves their instructions.
 #include "common.cuh"
 
 namespace tdm {
@@ -153,6 +154,10 @@ __device__ __forceinline__ float sqrt_approx(float x) {
     return r;
 }
 
+// Shared memory of one warp: B (the staged D first) at row stride kLd, V as
+// three columns of 64 (structure of arrays), and the row means of E.
+constexpr int kWarpFloats = kN * kLd + 3 * kN + kN;
+
 template <bool DIST>
 __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__restrict__ maps, int64_t n,
                                                                 float *__restrict__ coords,
@@ -161,19 +166,15 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                                                                 float *__restrict__ dist) {
     extern __shared__ __align__(16) float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float *sD = smem + warp * (kN * kLd);
-    // V as (c0, c1) pairs and c2 values: a broadcast 64-bit load is served
-    // per half warp and a 32-bit one per warp (3 wavefronts per row of V
-    // against 4 for a 128-bit broadcast)
-    float2 *sV01 = reinterpret_cast<float2 *>(smem + kMdsWarps * kN * kLd) + warp * kN * 2;
-    float *sV2 = reinterpret_cast<float *>(sV01 + kN);
-    float *sR = smem + kMdsWarps * kN * kLd + kMdsWarps * kN * 4 + warp * kN;
+    float *sE = smem + warp * kWarpFloats;
+    float *sV = sE + kN * kLd;     // v_c[64] for c = 0, 1, 2
+    float *sR = sV + 3 * kN;       // row means of E, negated
     const int i0 = lane, i1 = lane + 32;
 
     for (int64_t m = (int64_t)blockIdx.x * kMdsWarps + warp; m < n; m += (int64_t)gridDim.x * kMdsWarps) {
         const float *D = maps + m * kMapFloats;
         {   // the map into shared memory by 16-byte asynchronous copies, all in flight at once
-            const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(sD));
+            const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(sE));
 #pragma unroll
             for (int it = 0; it < 32; ++it) {
                 const int idx = it * 32 + lane;
@@ -186,69 +187,71 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         }
         __syncwarp();
 
-        // e_ij = D_ij + D_ji (twice the symmetric part); S = (e/2)^2, so
-        // B = -1/2 J S J = -1/8 J (e*e) J.  Lane l forms e*e of rows i0 and
-        // i1 in registers from row reads (float4) and column reads (lane l
-        // reads column l or l+32 of row j: consecutive words), all before any
-        // write, so no element is overwritten while another lane reads it.
-        float t0[kN], t1[kN];
-        float rs0 = 0.0f, rs1 = 0.0f;
+        // e_ij = D_ij + D_ji (twice the symmetric part) and E = e*e, so that
+        // B = -1/2 J (e/2)^2 J = -1/8 J E J.  Lane l forms rows i0 and i1 of E
+        // from row reads (float4) and column reads (lane l reads column l or
+        // l+32 of row j: consecutive words), as column pairs (2p, 2p+1) in
+        // packed float32, all before any write.  E is symmetric bit for bit,
+        // since e_ij and e_ji are the same sum.
+        float2 t0[kN / 2], t1[kN / 2];
+        float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j4 = 0; j4 < kN / 4; ++j4) {
-            const float4 a = *reinterpret_cast<const float4 *>(sD + i0 * kLd + 4 * j4);
-            const float4 b = *reinterpret_cast<const float4 *>(sD + i1 * kLd + 4 * j4);
-            const float ra[4] = {a.x, a.y, a.z, a.w}, rb[4] = {b.x, b.y, b.z, b.w};
+            const float4 a = ld4(sE + i0 * kLd + 4 * j4);
+            const float4 b = ld4(sE + i1 * kLd + 4 * j4);
+            float ca[4], cb[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int j = 4 * j4 + u;
-                const float e0 = ra[u] + sD[j * kLd + i0], e1 = rb[u] + sD[j * kLd + i1];
-                t0[j] = e0 * e0;
-                t1[j] = e1 * e1;
+                ca[u] = sE[(4 * j4 + u) * kLd + i0];
+                cb[u] = sE[(4 * j4 + u) * kLd + i1];
             }
-            // row sums in the order of a float4 pass over the rows
-            rs0 += (t0[4 * j4] + t0[4 * j4 + 1]) + (t0[4 * j4 + 2] + t0[4 * j4 + 3]);
-            rs1 += (t1[4 * j4] + t1[4 * j4 + 1]) + (t1[4 * j4 + 2] + t1[4 * j4 + 3]);
+            const float2 ea = __fadd2_rn(make_float2(a.x, a.y), make_float2(ca[0], ca[1]));
+            const float2 eb = __fadd2_rn(make_float2(a.z, a.w), make_float2(ca[2], ca[3]));
+            const float2 fa = __fadd2_rn(make_float2(b.x, b.y), make_float2(cb[0], cb[1]));
+            const float2 fb = __fadd2_rn(make_float2(b.z, b.w), make_float2(cb[2], cb[3]));
+            t0[2 * j4] = __fmul2_rn(ea, ea);
+            t0[2 * j4 + 1] = __fmul2_rn(eb, eb);
+            t1[2 * j4] = __fmul2_rn(fa, fa);
+            t1[2 * j4 + 1] = __fmul2_rn(fb, fb);
+            rs0 = __fadd2_rn(rs0, __fadd2_rn(t0[2 * j4], t0[2 * j4 + 1]));
+            rs1 = __fadd2_rn(rs1, __fadd2_rn(t1[2 * j4], t1[2 * j4 + 1]));
         }
-        const float r0 = rs0 * (1.0f / kN), r1 = rs1 * (1.0f / kN);
+        const float r0 = (rs0.x + rs0.y) * (1.0f / kN), r1 = (rs1.x + rs1.y) * (1.0f / kN);
         const float gm = wsum(r0 + r1) * (1.0f / kN);
-        // exact power-of-two scale bringing the mean of e*e to O(1); undone on
+        // exact power-of-two scale bringing the mean of E to O(1); undone on
         // the eigenvalues
         int ex = 0;
         frexpf(gm, &ex);
         const float scale = gm > 0.0f && isfinite(gm) ? ldexpf(1.0f, -ex) : 1.0f;
         const float cs = -0.125f * scale;
-        sR[i0] = r0;
-        sR[i1] = r1;
+        sR[i0] = -r0;    // negated: a - r is the packed sum a + (-r), rounded as the difference
+        sR[i1] = -r1;
         __syncwarp();    // every lane's reads of D are done: rows of B may replace it
-        // double centring: B_ij = cs (e2_ij - r_i - r_j + g); row i0 of B is
-        // also kept in registers for the products
-        const float g0 = gm - r0, g1 = gm - r1;
-        float *b0 = t0;
+        // double centring B_ij = cs ((E_ij + g_i) - r_j), g_i = g - r_i, in
+        // packed pairs; row i0 of B stays in registers for the products.  The
+        // centring is explicit because B annihilates the ones vector to
+        // rounding: a basis vector that is rounding noise (the null direction
+        // of a planar or collinear map) then does no harm.
+        const float2 cs2 = make_float2(cs, cs);
+        const float2 g0 = make_float2(gm - r0, gm - r0), g1 = make_float2(gm - r1, gm - r1);
 #pragma unroll
         for (int j4 = 0; j4 < kN / 4; ++j4) {
-            const float4 rj = *reinterpret_cast<const float4 *>(sR + 4 * j4);
-            float4 a, b;
-            a.x = cs * ((t0[4 * j4] + g0) - rj.x);
-            a.y = cs * ((t0[4 * j4 + 1] + g0) - rj.y);
-            a.z = cs * ((t0[4 * j4 + 2] + g0) - rj.z);
-            a.w = cs * ((t0[4 * j4 + 3] + g0) - rj.w);
-            b.x = cs * ((t1[4 * j4] + g1) - rj.x);
-            b.y = cs * ((t1[4 * j4 + 1] + g1) - rj.y);
-            b.z = cs * ((t1[4 * j4 + 2] + g1) - rj.z);
-            b.w = cs * ((t1[4 * j4 + 3] + g1) - rj.w);
-            b0[4 * j4] = a.x;
-            b0[4 * j4 + 1] = a.y;
-            b0[4 * j4 + 2] = a.z;
-            b0[4 * j4 + 3] = a.w;
-            *reinterpret_cast<float4 *>(sD + i0 * kLd + 4 * j4) = a;
-            *reinterpret_cast<float4 *>(sD + i1 * kLd + 4 * j4) = b;
+            const float4 rj = ld4(sR + 4 * j4);
+            const float2 ra = make_float2(rj.x, rj.y), rb = make_float2(rj.z, rj.w);
+            t0[2 * j4] = __fmul2_rn(cs2, __fadd2_rn(__fadd2_rn(t0[2 * j4], g0), ra));
+            t0[2 * j4 + 1] = __fmul2_rn(cs2, __fadd2_rn(__fadd2_rn(t0[2 * j4 + 1], g0), rb));
+            const float2 c = __fmul2_rn(cs2, __fadd2_rn(__fadd2_rn(t1[2 * j4], g1), ra));
+            const float2 d = __fmul2_rn(cs2, __fadd2_rn(__fadd2_rn(t1[2 * j4 + 1], g1), rb));
+            st4(sE + i0 * kLd + 4 * j4, make_float4(t0[2 * j4].x, t0[2 * j4].y, t0[2 * j4 + 1].x, t0[2 * j4 + 1].y));
+            st4(sE + i1 * kLd + 4 * j4, make_float4(c.x, c.y, d.x, d.y));
         }
         __syncwarp();
 
-        // start basis: the columns of the kK largest diagonal entries
+        // start basis: the columns of the kK largest diagonal entries of B
+        // (the points farthest from the centroid)
         float v0[kK], v1[kK];
         {
-            float d0 = sD[i0 * kLd + i0], d1 = sD[i1 * kLd + i1];
+            float d0 = sE[i0 * kLd + i0], d1 = sE[i1 * kLd + i1];
 #pragma unroll
             for (int c = 0; c < kK; ++c) {
                 float bv = d0 >= d1 ? d0 : d1;
@@ -256,39 +259,46 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                 warp_argmax(bv, bi);
                 if (bi == i0) d0 = -INFINITY;
                 if (bi == i1) d1 = -INFINITY;
-                v0[c] = sD[bi * kLd + i0];     // B[i0][bi] = B[bi][i0]
-                v1[c] = sD[bi * kLd + i1];
+                v0[c] = sE[bi * kLd + i0];     // B[i0][bi] = B[bi][i0]
+                v1[c] = sE[bi * kLd + i1];
             }
         }
         orthonormalize(v0, v1);
-        sV01[i0] = make_float2(v0[0], v0[1]);
-        sV01[i1] = make_float2(v1[0], v1[1]);
-        sV2[i0] = v0[2];
-        sV2[i1] = v1[2];
+#pragma unroll
+        for (int c = 0; c < kK; ++c) {
+            sV[c * kN + i0] = v0[c];
+            sV[c * kN + i1] = v1[c];
+        }
 
         float th[kK] = {0.f, 0.f, 0.f};
         float u0[kK], u1[kK];
         bool conv = false;
-        const float *bh = sD + i1 * kLd;
+        const float *bh = sE + i1 * kLd;
         for (int it = 0; it < kMaxIt; ++it) {
             __syncwarp();
-            float w0[kK] = {0.f, 0.f, 0.f}, w1[kK] = {0.f, 0.f, 0.f};
+            // W = B V: row i0 of B from registers, row i1 from shared memory,
+            // V broadcast four rows at a time; even and odd columns accumulate
+            // in the two halves of a packed pair
+            float2 a0[kK], a1[kK];
+#pragma unroll
+            for (int c = 0; c < kK; ++c) a0[c] = a1[c] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int j4 = 0; j4 < kN / 4; ++j4) {
-                const float4 x1 = *reinterpret_cast<const float4 *>(bh + 4 * j4);
-                const float xb[4] = {x1.x, x1.y, x1.z, x1.w};
+                const float4 e1 = ld4(bh + 4 * j4);
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float2 v01 = sV01[4 * j4 + t];
-                    const float4 v = make_float4(v01.x, v01.y, sV2[4 * j4 + t], 0.0f);
-                    const float xa = b0[4 * j4 + t];
-                    w0[0] = fmaf(xa, v.x, w0[0]);
-                    w0[1] = fmaf(xa, v.y, w0[1]);
-                    w0[2] = fmaf(xa, v.z, w0[2]);
-                    w1[0] = fmaf(xb[t], v.x, w1[0]);
-                    w1[1] = fmaf(xb[t], v.y, w1[1]);
-                    w1[2] = fmaf(xb[t], v.z, w1[2]);
+                for (int c = 0; c < kK; ++c) {
+                    const float4 v = ld4(sV + c * kN + 4 * j4);
+                    a0[c] = __ffma2_rn(t0[2 * j4], make_float2(v.x, v.y), a0[c]);
+                    a0[c] = __ffma2_rn(t0[2 * j4 + 1], make_float2(v.z, v.w), a0[c]);
+                    a1[c] = __ffma2_rn(make_float2(e1.x, e1.y), make_float2(v.x, v.y), a1[c]);
+                    a1[c] = __ffma2_rn(make_float2(e1.z, e1.w), make_float2(v.z, v.w), a1[c]);
                 }
+            }
+            float w0[kK], w1[kK];
+#pragma unroll
+            for (int c = 0; c < kK; ++c) {
+                w0[c] = a0[c].x + a0[c].y;
+                w1[c] = a1[c].x + a1[c].y;
             }
             // Rayleigh quotient H = V^T B V (symmetrised)
             float H[kK][kK];
@@ -303,6 +313,7 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                 }
             float Y[kK][kK];
             eig3(H, Y, th);
+            // Ritz vectors U = V Y and B U = W Y
             float bu0[kK], bu1[kK];
 #pragma unroll
             for (int c = 0; c < kK; ++c) {
@@ -334,10 +345,11 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                 v1[c] = bu1[c];
             }
             __syncwarp();
-            sV01[i0] = make_float2(v0[0], v0[1]);
-            sV01[i1] = make_float2(v1[0], v1[1]);
-            sV2[i0] = v0[2];
-            sV2[i1] = v1[2];
+#pragma unroll
+            for (int c = 0; c < kK; ++c) {
+                sV[c * kN + i0] = v0[c];
+                sV[c * kN + i1] = v1[c];
+            }
         }
         {   // the warp's next map into L2 while this one's coordinates and
             // distances are written (issued at the start of the map, or before
@@ -351,39 +363,62 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         if (!conv && lane == 0) atomicOr(flags, (uint32_t)TDM_FLAG_MDS_NOT_CONVERGED);
 
         const float inv_scale = 1.0f / scale;
-        float *X = coords + m * (kN * 3);
+        float x0[kK], x1[kK];
 #pragma unroll
         for (int c = 0; c < kK; ++c) {
             const float sq = sqrtf(fmaxf(th[c], 0.0f) * inv_scale);
-            X[i0 * 3 + c] = u0[c] * sq;
-            X[i1 * 3 + c] = u1[c] * sq;
+            x0[c] = u0[c] * sq;
+            x1[c] = u1[c] * sq;
+        }
+        float *X = coords + m * (kN * 3);
+#pragma unroll
+        for (int c = 0; c < kK; ++c) {
+            X[i0 * 3 + c] = x0[c];
+            X[i1 * 3 + c] = x1[c];
         }
         if (eig != nullptr && lane < 3) eig[m * 3 + lane] = (lane == 0 ? th[0] : lane == 1 ? th[1] : th[2]) * inv_scale;
         if (DIST) {
-            // the distance map of the coordinates, as pdist_kernel computes it:
-            // the coordinates go to shared memory (the V arrays are free now),
-            // then row r is written by the whole warp, two columns per lane,
-            // with coalesced 8-byte streaming stores
-            float *sc = reinterpret_cast<float *>(sV01);    // x[64], y[64], z[64]
+            // the distance map of the coordinates, as pdist_kernel computes it.
+            // The coordinates go to shared memory twice: as x[64], y[64], z[64]
+            // for the columns (in the V arrays) and, for the rows, as the packed
+            // pairs (x, x, y, y) and (z, z) of each bead (in the E area, free
+            // now).  Lanes 0-15 write row 2p and lanes 16-31 row 2p+1, four
+            // columns per lane, with 16-byte streaming stores.
+            float4 *sb = reinterpret_cast<float4 *>(sE);
+            float2 *sz = reinterpret_cast<float2 *>(sE + 4 * kN);
             __syncwarp();
 #pragma unroll
             for (int c = 0; c < kK; ++c) {
-                const float sq = sqrtf(fmaxf(th[c], 0.0f) * inv_scale);
-                sc[c * kN + i0] = u0[c] * sq;
-                sc[c * kN + i1] = u1[c] * sq;
+                sV[c * kN + i0] = x0[c];
+                sV[c * kN + i1] = x1[c];
             }
+            sb[i0] = make_float4(x0[0], x0[0], x0[1], x0[1]);
+            sb[i1] = make_float4(x1[0], x1[0], x1[1], x1[1]);
+            sz[i0] = make_float2(x0[2], x0[2]);
+            sz[i1] = make_float2(x1[2], x1[2]);
             __syncwarp();
-            const float2 cx = reinterpret_cast<const float2 *>(sc)[lane];
-            const float2 cy = reinterpret_cast<const float2 *>(sc + kN)[lane];
-            const float2 cz = reinterpret_cast<const float2 *>(sc + 2 * kN)[lane];
-            float2 *out = reinterpret_cast<float2 *>(dist + m * kMapFloats) + lane;
-#pragma unroll 8
-            for (int row = 0; row < kN; ++row) {
-                const float xi = sc[row], yi = sc[kN + row], zi = sc[2 * kN + row];
-                float2 d;
-                d.x = sqrt_approx(fmaf(zi - cz.x, zi - cz.x, fmaf(yi - cy.x, yi - cy.x, (xi - cx.x) * (xi - cx.x))));
-                d.y = sqrt_approx(fmaf(zi - cz.y, zi - cz.y, fmaf(yi - cy.y, yi - cy.y, (xi - cx.y) * (xi - cx.y))));
-                __stcs(out + row * (kN / 2), d);
+            const int q = lane & 15, h = lane >> 4;
+            const float4 cx = ld4(sV + 4 * q), cy = ld4(sV + kN + 4 * q), cz = ld4(sV + 2 * kN + 4 * q);
+            const float2 nx01 = make_float2(-cx.x, -cx.y), nx23 = make_float2(-cx.z, -cx.w);
+            const float2 ny01 = make_float2(-cy.x, -cy.y), ny23 = make_float2(-cy.z, -cy.w);
+            const float2 nz01 = make_float2(-cz.x, -cz.y), nz23 = make_float2(-cz.z, -cz.w);
+            float4 *out = reinterpret_cast<float4 *>(dist + m * kMapFloats) + h * (kN / 4) + q;
+#pragma unroll 4
+            for (int rp = 0; rp < kN / 2; ++rp) {
+                const int row = 2 * rp + h;
+                const float4 bxy = sb[row];
+                const float2 bz = sz[row];
+                const float2 xx = make_float2(bxy.x, bxy.y), yy = make_float2(bxy.z, bxy.w);
+                const float2 dx01 = __fadd2_rn(xx, nx01), dx23 = __fadd2_rn(xx, nx23);
+                const float2 dy01 = __fadd2_rn(yy, ny01), dy23 = __fadd2_rn(yy, ny23);
+                const float2 dz01 = __fadd2_rn(bz, nz01), dz23 = __fadd2_rn(bz, nz23);
+                float2 s01 = __fmul2_rn(dx01, dx01), s23 = __fmul2_rn(dx23, dx23);
+                s01 = __ffma2_rn(dy01, dy01, s01);
+                s23 = __ffma2_rn(dy23, dy23, s23);
+                s01 = __ffma2_rn(dz01, dz01, s01);
+                s23 = __ffma2_rn(dz23, dz23, s23);
+                __stcs(out + rp * (kN / 2),
+                       make_float4(sqrt_approx(s01.x), sqrt_approx(s01.y), sqrt_approx(s23.x), sqrt_approx(s23.y)));
             }
         }
         __syncwarp();
@@ -443,8 +478,9 @@ int sms() {
 cudaError_t launch_mds(const float *maps, int64_t n, float *coords, float *eigvals, uint32_t *flags, float *dist,
                        cudaStream_t st) {
     if (n <= 0) return cudaSuccess;
-    const size_t smem = sizeof(float) * (size_t)kMdsWarps * (kN * kLd + kN * 4 + kN);
-    static_assert((kMdsWarps * kN * kLd * sizeof(float)) % 16 == 0, "float4 alignment of the V tiles");
+    const size_t smem = sizeof(float) * (size_t)kMdsWarps * kWarpFloats;
+    static_assert((kWarpFloats * sizeof(float)) % 16 == 0 && (kN * kLd * sizeof(float)) % 16 == 0,
+                  "float4 alignment of every warp's E and V tiles");
     const void *kern = dist != nullptr ? reinterpret_cast<const void *>(mds_kernel<true>)
                                        : reinterpret_cast<const void *>(mds_kernel<false>);
     LaunchShape shape;
