@@ -68,6 +68,52 @@ __device__ __forceinline__ void orthonormalize(float (&a0)[kK], float (&a1)[kK])
     }
 }
 
+// Orthonormalises the kK columns Y (rows (l, l+32) per lane) whose Gram
+// matrix G = Y^T Y is given: Y diag(s) is nearly orthonormal when the columns
+// are nearly orthogonal, whatever their scale, and Cholesky QR of the scaled
+// Gram matrix (a 3 x 3 factorisation done by every lane) then needs no further
+// reduction.  A column whose norm or pivot vanishes becomes zero, as in
+// orthonormalize.  Returns the largest off-diagonal of the scaled Gram matrix,
+// a measure of how far from orthogonal the columns were.
+__device__ __forceinline__ float cholqr(float (&a0)[kK], float (&a1)[kK], const float (&G)[kK][kK]) {
+    float sc[kK];
+#pragma unroll
+    for (int c = 0; c < kK; ++c) sc[c] = G[c][c] > 1e-37f ? rsqrt_approx(G[c][c]) : 0.0f;
+    const float g01 = G[0][1] * sc[0] * sc[1], g02 = G[0][2] * sc[0] * sc[2], g12 = G[1][2] * sc[1] * sc[2];
+    const float g00 = G[0][0] * sc[0] * sc[0], g11 = G[1][1] * sc[1] * sc[1], g22 = G[2][2] * sc[2] * sc[2];
+    // G' = L L^T; the new columns are Y diag(sc) L^-T, by forward substitution
+    const float p0 = g00;
+    const float i0 = p0 > 1e-12f ? rsqrt_approx(p0) : 0.0f;
+    const float l10 = g01 * i0, l20 = g02 * i0;
+    const float p1 = fmaf(-l10, l10, g11);
+    const float i1 = p1 > 1e-12f ? rsqrt_approx(p1) : 0.0f;
+    const float l21 = fmaf(-l20, l10, g12) * i1;
+    const float p2 = fmaf(-l21, l21, fmaf(-l20, l20, g22));
+    const float i2 = p2 > 1e-12f ? rsqrt_approx(p2) : 0.0f;
+    const float y0a = a0[0] * sc[0], y0b = a1[0] * sc[0];
+    const float y1a = a0[1] * sc[1], y1b = a1[1] * sc[1];
+    const float y2a = a0[2] * sc[2], y2b = a1[2] * sc[2];
+    a0[0] = y0a * i0;
+    a1[0] = y0b * i0;
+    a0[1] = fmaf(-l10, a0[0], y1a) * i1;
+    a1[1] = fmaf(-l10, a1[0], y1b) * i1;
+    a0[2] = fmaf(-l21, a0[1], fmaf(-l20, a0[0], y2a)) * i2;
+    a1[2] = fmaf(-l21, a1[1], fmaf(-l20, a1[0], y2b)) * i2;
+    return fmaxf(fabsf(g01), fmaxf(fabsf(g02), fabsf(g12)));
+}
+
+// The Gram matrix of the kK columns (rows (l, l+32) per lane), reduced over the warp.
+__device__ __forceinline__ void gram(const float (&a0)[kK], const float (&a1)[kK], float (&G)[kK][kK]) {
+#pragma unroll
+    for (int a = 0; a < kK; ++a)
+#pragma unroll
+        for (int b = a; b < kK; ++b) {
+            const float g = wsum(fmaf(a0[a], a0[b], a1[a] * a1[b]));
+            G[a][b] = g;
+            G[b][a] = g;
+        }
+}
+
 // One Jacobi rotation zeroing H[P][Q] of the symmetric kK x kK H (both
 // halves kept), accumulated into Y (Golub & Van Loan §8.5: the symmetric 2 x 2
 // Schur step, with the diagonal updated by t * H[P][Q]).
@@ -326,19 +372,28 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                     bu1[c] = fmaf(w1[a], Y[a][c], bu1[c]);
                 }
             }
-            float rmax = 0.0f;
+            // the Ritz residuals and the Gram matrix of B U, reduced together:
+            // B U = U Theta + R with R orthogonal to U, so its columns are
+            // nearly orthogonal whatever their scale, and one Cholesky QR of
+            // the scaled Gram matrix orthonormalises them (a second pass runs
+            // when they were not)
+            float rmax = 0.0f, G[kK][kK];
 #pragma unroll
             for (int c = 0; c < kK; ++c) {
                 const float e0 = fmaf(-th[c], u0[c], bu0[c]);
                 const float e1 = fmaf(-th[c], u1[c], bu1[c]);
                 rmax = fmaxf(rmax, wsum(fmaf(e0, e0, e1 * e1)));
             }
+            gram(bu0, bu1, G);
             const float lim = kTol * fabsf(th[0]);
             if (rmax <= lim * lim) {
                 conv = true;
                 break;
             }
-            orthonormalize(bu0, bu1);
+            if (cholqr(bu0, bu1, G) > 1e-2f) {
+                gram(bu0, bu1, G);
+                cholqr(bu0, bu1, G);
+            }
 #pragma unroll
             for (int c = 0; c < kK; ++c) {
                 v0[c] = bu0[c];
