@@ -35,7 +35,7 @@ def _run(tdm, X, T, overlap):
 @pytest.mark.parametrize("C,T,B,o,noise", [(2, 5, 3, 12, 0.05), (1, 32, 8, 12, 0.02), (2, 40, 3, 8, 0.05),
                                            (1, 3, 2, 32, 0.0), (3, 1, 2, 12, 0.0), (2, 6, 3, 7, 0.05),
                                            (1, 4, 5, 5, 0.0), (1, 33, 2, 12, 0.05), (1, 64, 2, 32, 0.05),
-                                           (2, 65, 2, 8, 0.0)])
+                                           (2, 65, 2, 12, 0.0)])
 def test_stitch_matches_oracle(tdm, C, T, B, o, noise):
     # tiles go through the kernel 32 at a time: T = 32, 33, 40, 64 and 65 put
     # a chunk boundary at the end, before a single tile, inside, between two

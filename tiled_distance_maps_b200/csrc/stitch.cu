@@ -80,18 +80,25 @@ __device__ __forceinline__ float rsqrt_approx(float x) {
     return r;
 }
 
-// Eigen-decomposition of a symmetric 3 x 3 matrix by cyclic Jacobi (Golub &
-// Van Loan §8.5); descending eigenvalues, eigenvectors in the columns of V.
-// The rotation's reciprocals and square roots are the hardware approximations
-// (a few ulp): the rotation stays orthogonal to float32 rounding, and the skip
-// test below keeps theta^2 finite (|theta| < 5e11).
+// Eigen-decomposition of a symmetric positive semidefinite 3 x 3 matrix by
+// cyclic Jacobi (Golub & Van Loan §8.5); descending eigenvalues, eigenvectors
+// in the columns of V.  An off-diagonal entry counts as zero when
+// a_pq^2 <= 1e-14 a_pp a_qq, relative to its own two diagonal entries: a
+// test relative to the whole diagonal would leave the eigenvectors of the
+// small eigenvalues of an elongated overlap (M^T M squares its condition)
+// rotated by about 1e-6 l_1 / gap.  The matrix is scaled by its trace first,
+// so no product overflows.  The rotation's reciprocals and square roots are
+// the hardware approximations (a few ulp): the rotation stays orthogonal to
+// float32 rounding.
 template <int P, int Q>
 __device__ __forceinline__ void jrot3(float (&A)[3][3], float (&V)[3][3]) {
     const float apq = A[P][Q];
-    if (!(fabsf(apq) > 1e-12f * (fabsf(A[P][P]) + fabsf(A[Q][Q])))) return;
+    if (!(apq * apq > 1e-14f * (A[P][P] * A[Q][Q]))) return;
     const float theta = (A[Q][Q] - A[P][P]) * 0.5f * rcp_approx(apq);
+    const float at = fabsf(theta);
+    // t = sign(theta) / (|theta| + sqrt(theta^2 + 1)), 1 / (2 theta) where theta^2 would overflow
     const float r2 = fmaf(theta, theta, 1.0f);
-    const float t = copysignf(rcp_approx(fabsf(theta) + r2 * rsqrt_approx(r2)), theta);
+    const float t = copysignf(at > 1e18f ? 0.5f * rcp_approx(at) : rcp_approx(at + r2 * rsqrt_approx(r2)), theta);
     const float c = rsqrt_approx(fmaf(t, t, 1.0f));
     const float s = t * c;
     A[P][P] = fmaf(-t, apq, A[P][P]);
@@ -114,10 +121,17 @@ __device__ __forceinline__ void sym_eig3(float (&A)[3][3], float (&V)[3][3], flo
     for (int i = 0; i < 3; ++i)
 #pragma unroll
         for (int j = 0; j < 3; ++j) V[i][j] = i == j ? 1.0f : 0.0f;
+    const float tr = A[0][0] + A[1][1] + A[2][2];
+    const float sc = tr > 1e-37f ? rcp_approx(tr) : 1.0f;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+        for (int j = 0; j < 3; ++j) A[i][j] *= sc;
     for (int sweep = 0; sweep < 16; ++sweep) {
-        const float off = A[0][1] * A[0][1] + A[0][2] * A[0][2] + A[1][2] * A[1][2];
-        const float dia = A[0][0] * A[0][0] + A[1][1] * A[1][1] + A[2][2] * A[2][2];
-        if (off <= 1e-12f * dia) break;    // off-diagonal within 1e-6 of the diagonal (float32 reaches no further)
+        if (!(A[0][1] * A[0][1] > 1e-14f * (A[0][0] * A[1][1])) &&
+            !(A[0][2] * A[0][2] > 1e-14f * (A[0][0] * A[2][2])) &&
+            !(A[1][2] * A[1][2] > 1e-14f * (A[1][1] * A[2][2])))
+            break;
         jrot3<0, 1>(A, V);
         jrot3<0, 2>(A, V);
         jrot3<1, 2>(A, V);
@@ -143,38 +157,11 @@ __device__ __forceinline__ void sym_eig3(float (&A)[3][3], float (&V)[3][3], flo
             }
 }
 
-// Rigid map of tile k+1 onto tile k over the o overlap beads and its RMSD.
-__device__ Rigid align_seam(const float *P, const float *Q, int o, float *rmsd) {
-    float pc[3] = {0.f, 0.f, 0.f}, qc[3] = {0.f, 0.f, 0.f};
-    for (int i = 0; i < o; ++i)
-#pragma unroll
-        for (int d = 0; d < 3; ++d) {
-            pc[d] += P[3 * i + d];
-            qc[d] += Q[3 * i + d];
-        }
-    const float inv_o = 1.0f / (float)o;
-#pragma unroll
-    for (int d = 0; d < 3; ++d) {
-        pc[d] *= inv_o;
-        qc[d] *= inv_o;
-    }
-    // M = sum_i (p_i - pc)(q_i - qc)^T
-    float M[3][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
-    for (int i = 0; i < o; ++i) {
-        float p[3], q[3];
-#pragma unroll
-        for (int d = 0; d < 3; ++d) {
-            p[d] = P[3 * i + d] - pc[d];
-            q[d] = Q[3 * i + d] - qc[d];
-        }
-#pragma unroll
-        for (int a = 0; a < 3; ++a)
-#pragma unroll
-            for (int b = 0; b < 3; ++b) M[a][b] = fmaf(p[a], q[b], M[a][b]);
-    }
-    // polar factor R = U V^T of M = U S V^T: V from the eigenvectors of M^T M,
-    // U = M V S^-1 re-orthonormalised (third column completed by the cross
-    // product when M is rank deficient)
+// Polar factor R = U V^T of M = U S V^T through the eigenvectors V of M^T M:
+// U = M V S^-1 re-orthonormalised, its third column completed by the cross
+// product when M is rank deficient (an overlap of 3 beads, or coplanar ones).
+// The fallback of newton_polar.
+__device__ __noinline__ void polar_by_eig(const float (&M)[3][3], float (&R)[9]) {
     float A[3][3], V[3][3], lam[3];
 #pragma unroll
     for (int a = 0; a < 3; ++a)
@@ -212,16 +199,128 @@ __device__ Rigid align_seam(const float *P, const float *Q, int o, float *rmsd) 
         U[1][2] = U[2][0] * U[0][1] - U[0][0] * U[2][1];
         U[2][2] = U[0][0] * U[1][1] - U[1][0] * U[0][1];
     }
-    Rigid g;
 #pragma unroll
     for (int a = 0; a < 3; ++a)
 #pragma unroll
-        for (int b = 0; b < 3; ++b) g.r[3 * a + b] = U[a][0] * V[b][0] + U[a][1] * V[b][1] + U[a][2] * V[b][2];
+        for (int b = 0; b < 3; ++b) R[3 * a + b] = U[a][0] * V[b][0] + U[a][1] * V[b][1] + U[a][2] * V[b][2];
+}
+
+// Polar factor of M by the scaled Newton iteration X <- (g X + X^-T / g) / 2,
+// g = (|X^-1|_F / |X|_F)^(1/2) (Higham, "Computing the polar decomposition --
+// with applications", 1986), from X = M / |M|_F.  It works on M itself, so
+// the condition of M is not squared as in M^T M, and it converges to the
+// orthogonal factor whatever the sign of det M (an improper R is wanted:
+// recovered coordinates are defined up to reflection).  X^-T is the cofactor
+// matrix over the determinant.  Returns false, leaving R alone, when M is
+// nearly singular (|det X| < 1e-6) or the iteration has not settled after 12
+// steps; the caller then takes polar_by_eig.
+__device__ __forceinline__ bool newton_polar(const float (&M)[3][3], float (&R)[9]) {
+    float X[9], nx = 0.0f;
+#pragma unroll
+    for (int a = 0; a < 9; ++a) {
+        X[a] = M[a / 3][a % 3];
+        nx = fmaf(X[a], X[a], nx);
+    }
+    if (!(nx > 1e-37f)) return false;
+    const float inx = rsqrt_approx(nx);
+#pragma unroll
+    for (int a = 0; a < 9; ++a) X[a] *= inx;
+    nx = 1.0f;
+    for (int it = 0; it < 12; ++it) {
+        float Cf[9];
+        Cf[0] = fmaf(X[4], X[8], -X[5] * X[7]);
+        Cf[1] = fmaf(X[5], X[6], -X[3] * X[8]);
+        Cf[2] = fmaf(X[3], X[7], -X[4] * X[6]);
+        Cf[3] = fmaf(X[2], X[7], -X[1] * X[8]);
+        Cf[4] = fmaf(X[0], X[8], -X[2] * X[6]);
+        Cf[5] = fmaf(X[1], X[6], -X[0] * X[7]);
+        Cf[6] = fmaf(X[1], X[5], -X[2] * X[4]);
+        Cf[7] = fmaf(X[2], X[3], -X[0] * X[5]);
+        Cf[8] = fmaf(X[0], X[4], -X[1] * X[3]);
+        const float det = fmaf(X[0], Cf[0], fmaf(X[1], Cf[1], X[2] * Cf[2]));
+        if (it == 0 && !(fabsf(det) > 1e-6f)) return false;
+        const float rd = rcp_approx(det);
+        float ny = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 9; ++a) {
+            Cf[a] *= rd;                       // X^-T
+            ny = fmaf(Cf[a], Cf[a], ny);
+        }
+        // g = (ny / nx)^(1/4); X <- (g/2) X + (1/(2g)) X^-T
+        const float g = rsqrt_approx(rsqrt_approx(ny * rcp_approx(nx)));
+        const float ha = 0.5f * g, hb = 0.5f * rcp_approx(g);
+        float dmax = 0.0f, nn = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 9; ++a) {
+            const float xn = fmaf(ha, X[a], hb * Cf[a]);
+            dmax = fmaxf(dmax, fabsf(xn - X[a]));
+            X[a] = xn;
+            nn = fmaf(xn, xn, nn);
+        }
+        nx = nn;
+        if (dmax <= 1e-6f) {
+#pragma unroll
+            for (int a = 0; a < 9; ++a) R[a] = X[a];
+            return true;
+        }
+    }
+    return false;
+}
+
+// Rigid map of tile k+1 onto tile k over the o overlap beads and its RMSD.
+// The beads are visited from bead `rot` on (cyclically), so that lanes which
+// read their own seams at a common stride spread over the banks.  The cross-
+// covariance is formed in one pass from offsets to the first bead visited:
+// M = sum (dp_i)(dq_i)^T - o m_p m_q^T, with m the mean offsets, which keeps
+// its terms near the overlap's own extent however far the tiles sit from the
+// origin.
+__device__ Rigid align_seam(const float *P, const float *Q, int o, int rot, float *rmsd) {
+    float pr[3], qr[3];
+    const int i0 = rot % o;
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+        pr[d] = P[3 * i0 + d];
+        qr[d] = Q[3 * i0 + d];
+    }
+    float sp[3] = {0.f, 0.f, 0.f}, sq[3] = {0.f, 0.f, 0.f};
+    float M[3][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+    int i = i0;
+    for (int n = 0; n < o; ++n) {
+        float dp[3], dq[3];
+#pragma unroll
+        for (int d = 0; d < 3; ++d) {
+            dp[d] = P[3 * i + d] - pr[d];
+            dq[d] = Q[3 * i + d] - qr[d];
+            sp[d] += dp[d];
+            sq[d] += dq[d];
+        }
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int b = 0; b < 3; ++b) M[a][b] = fmaf(dp[a], dq[b], M[a][b]);
+        if (++i == o) i = 0;
+    }
+    const float inv_o = 1.0f / (float)o;
+    float pc[3], qc[3];
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+        sp[d] *= inv_o;
+        sq[d] *= inv_o;
+        pc[d] = pr[d] + sp[d];
+        qc[d] = qr[d] + sq[d];
+    }
+#pragma unroll
+    for (int a = 0; a < 3; ++a)
+#pragma unroll
+        for (int b = 0; b < 3; ++b) M[a][b] = fmaf(-(float)o * sp[a], sq[b], M[a][b]);
+    Rigid g;
+    if (!newton_polar(M, g.r)) polar_by_eig(M, g.r);
 #pragma unroll
     for (int a = 0; a < 3; ++a)
         g.t[a] = pc[a] - (g.r[3 * a] * qc[0] + g.r[3 * a + 1] * qc[1] + g.r[3 * a + 2] * qc[2]);
     float ss = 0.0f;
-    for (int i = 0; i < o; ++i) {
+    i = i0;
+    for (int n = 0; n < o; ++n) {
         float y[3];
         apply(g, Q + 3 * i, y);
 #pragma unroll
@@ -229,6 +328,7 @@ __device__ Rigid align_seam(const float *P, const float *Q, int o, float *rmsd) 
             const float e = y[d] - P[3 * i + d];
             ss = fmaf(e, e, ss);
         }
+        if (++i == o) i = 0;
     }
     *rmsd = sqrtf(ss * inv_o);
     return g;
@@ -247,7 +347,7 @@ __device__ __forceinline__ Rigid chunk_maps(const float *P, const float *Q, int 
     Rigid tk = identity();    // seam k: tile k+1 onto tile k
     if (k < T - 1) {
         float r;
-        tk = align_seam(P, Q, o, &r);
+        tk = align_seam(P, Q, o, lane, &r);
         if (resid != nullptr) resid[pair * (T - 1) + k] = r;
     }
     Rigid sk = tk;    // inclusive scan: t_{k0} o ... o t_k
@@ -262,14 +362,6 @@ __device__ __forceinline__ Rigid chunk_maps(const float *P, const float *Q, int 
     carry_prev = shfl_idx(gk, 31);
     carry = shfl_idx(gnext, 31);
     return gk;
-}
-
-// 4-byte asynchronous global -> shared copy (a chunk's copies are all in
-// flight before the CTA waits for them)
-__device__ __forceinline__ void async_copy4(float *dst, const float *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src)
-                 : "memory");
 }
 
 __device__ __forceinline__ Rigid smem_map(const Rigid *g) {
@@ -292,37 +384,97 @@ __device__ __forceinline__ void smem_store_map(Rigid *g, const Rigid &m) {
 constexpr int kStitchThreads = 128;
 constexpr int kChunk = 32;                 // seams aligned per chunk, a lane each
 constexpr int kSlots = kChunk + 1;         // tiles staged per chunk: its 32 and the next
-constexpr int kTileLd = kN * 3 + 1;        // 193 floats: odd, so the lanes' reads of their seams do not conflict
+constexpr int kTileLd = kN * 3 + 4;        // 196 floats: 16-byte rows; lane k's seam reads rotate by k beads
 // shared memory: the maps of the chunk's tiles and of the tile before it, the
 // staged tiles, and the last o beads of the tile before the chunk
 constexpr int kMapsFloats = (kSlots + 1) * 12;
 constexpr int kStitchSmemFloats = kMapsFloats + kSlots * kTileLd + 96;
 
+// x / d for 0 <= x < 2^31 and 0 < d < 2^16 by the multiply-shift of m = ceil(2^32 / d)
+__device__ __forceinline__ int div_by(int x, int d, uint32_t m) {
+    int k = (int)(((uint64_t)(uint32_t)x * m) >> 32);
+    if (k * d > x) --k;
+    return k;
+}
+
+// G chain beads of tile k from bead j on (G = 4: 12 floats, 16-byte aligned in
+// the staged tile, the previous tile's copy and the chain; G = 1 otherwise):
+// the tile's aligned copy, averaged with tile k-1's over the overlap.
+template <int G>
+__device__ __forceinline__ void place_beads(const float *tile, const float *prev, const Rigid *gk, const Rigid *gp,
+                                            bool ov, float *dst) {
+    float x[3 * G], y[3 * G];
+    if constexpr (G == 4) {
+#pragma unroll
+        for (int v = 0; v < 3; ++v) *reinterpret_cast<float4 *>(x + 4 * v) = reinterpret_cast<const float4 *>(tile)[v];
+    } else {
+#pragma unroll
+        for (int v = 0; v < 3; ++v) x[v] = tile[v];
+    }
+    const Rigid g = smem_map(gk);
+#pragma unroll
+    for (int u = 0; u < G; ++u) apply(g, x + 3 * u, y + 3 * u);
+    if (ov) {
+        float xp[3 * G];
+        if constexpr (G == 4) {
+#pragma unroll
+            for (int v = 0; v < 3; ++v)
+                *reinterpret_cast<float4 *>(xp + 4 * v) = reinterpret_cast<const float4 *>(prev)[v];
+        } else {
+#pragma unroll
+            for (int v = 0; v < 3; ++v) xp[v] = prev[v];
+        }
+        const Rigid h = smem_map(gp);
+#pragma unroll
+        for (int u = 0; u < G; ++u) {
+            float y1[3];
+            apply(h, xp + 3 * u, y1);
+#pragma unroll
+            for (int d = 0; d < 3; ++d) y[3 * u + d] = 0.5f * (y1[d] + y[3 * u + d]);
+        }
+    }
+    if constexpr (G == 4) {
+#pragma unroll
+        for (int v = 0; v < 3; ++v) reinterpret_cast<float4 *>(dst)[v] = *reinterpret_cast<const float4 *>(y + 4 * v);
+    } else {
+#pragma unroll
+        for (int v = 0; v < 3; ++v) dst[v] = y[v];
+    }
+}
+
 // One CTA per (chain, sample) pair.  Tile k owns chain positions [k s, k s + s),
 // the last tile [k s, k s + 64); the first o beads of tile k > 0 are the mean of
-// tile k-1's and tile k's aligned copies.  Bit for bit the arithmetic of the
-// alignment (align_seam), the scan (chunk_maps) and the placement (apply, then
-// the mean) does not depend on the chunking.
+// tile k-1's and tile k's aligned copies.  The arithmetic does not depend on
+// the chunking.  G = 4 beads per thread needs o % 4 == 0 (four beads then stay
+// in one tile and on one side of the overlap boundary, 16-byte aligned).
+template <int G>
 __global__ void __launch_bounds__(kStitchThreads, 7) stitch_kernel(const float *__restrict__ coords, int T, int B,
                                                                    int o, float *__restrict__ chain,
                                                                    float *__restrict__ resid) {
     extern __shared__ __align__(16) float sm[];
-    Rigid *smaps = reinterpret_cast<Rigid *>(sm);           // [0, 32]: tiles k0 .. k0+31; [32]: tile k0-1
-    float *stile = sm + kMapsFloats;                         // [33][193]: tiles k0 .. k0+32
+    Rigid *smaps = reinterpret_cast<Rigid *>(sm);           // [0, 32): tiles k0 .. k0+31; [32]: tile k0-1
+    float *stile = sm + kMapsFloats;                         // [33][196]: tiles k0 .. k0+32
     float *sprev = stile + kSlots * kTileLd;                 // tile k0-1's beads s .. 63
     const int64_t pair = blockIdx.x;
     const int c = (int)(pair / B), b = (int)(pair - (int64_t)(pair / B) * B);
     const int s = kN - o;
     const int L = kN + (T - 1) * s;
     const int tid = threadIdx.x;
+    const int gpt = s / G;                                   // bead groups per tile stride
+    const uint32_t mg = (uint32_t)((0x100000000ULL + (uint64_t)gpt - 1) / (uint64_t)gpt);
     float *dst = chain + pair * (int64_t)L * 3;
     Rigid carry = identity(), carry_prev = identity();       // warp 0: G_{k0}, G_{k0-1}
     for (int k0 = 0; k0 < T; k0 += kChunk) {
         const int nt = min(kSlots, T - k0);                  // tiles staged
         const int nc = min(kChunk, T - k0);                  // tiles placed
-        for (int i = 0; i < nt; ++i) {
-            const float *src = coords + (((int64_t)c * T + k0 + i) * B + b) * (kN * 3);
-            for (int e = tid; e < kN * 3; e += kStitchThreads) async_copy4(stile + i * kTileLd + e, src + e);
+        // 16-byte copies: 48 per tile
+        for (int idx = tid; idx < nt * 48; idx += kStitchThreads) {
+            const int i = idx / 48, e = idx - i * 48;
+            const float *src = coords + (((int64_t)c * T + k0 + i) * B + b) * (kN * 3) + 4 * e;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(
+                             __cvta_generic_to_shared(stile + i * kTileLd + 4 * e))),
+                         "l"(src)
+                         : "memory");
         }
         asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
         __syncthreads();
@@ -334,29 +486,17 @@ __global__ void __launch_bounds__(kStitchThreads, 7) stitch_kernel(const float *
             if (lane < nc) smem_store_map(smaps + lane, gk);
         }
         __syncthreads();
-        // the chunk's beads: nc * s of them, plus the last tile's o beyond its stride
-        const int nb = nc * s + (k0 + nc == T ? o : 0);
-        for (int idx = tid; idx < nb; idx += kStitchThreads) {
-            int kl = idx / s;
+        // the chunk's bead groups: nc tiles of s beads, plus the last tile's o
+        const int ng = nc * gpt + (k0 + nc == T ? o / G : 0);
+        for (int g = tid; g < ng; g += kStitchThreads) {
+            int kl = div_by(g, gpt, mg);
             if (kl > nc - 1) kl = nc - 1;
-            const int j = idx - kl * s;
+            const int j = (g - kl * gpt) * G;
             const int k = k0 + kl;
-            float x[3], y[3];
-#pragma unroll
-            for (int d = 0; d < 3; ++d) x[d] = stile[kl * kTileLd + 3 * j + d];
-            apply(smem_map(smaps + kl), x, y);
-            if (k > 0 && j < o) {
-                float xp[3], y1[3];
-                const float *bp = kl > 0 ? stile + (kl - 1) * kTileLd + 3 * (s + j) : sprev + 3 * j;
-#pragma unroll
-                for (int d = 0; d < 3; ++d) xp[d] = bp[d];
-                apply(smem_map(smaps + (kl > 0 ? kl - 1 : kChunk)), xp, y1);
-#pragma unroll
-                for (int d = 0; d < 3; ++d) y[d] = 0.5f * (y1[d] + y[d]);
-            }
-            float *out = dst + ((int64_t)k * s + j) * 3;
-#pragma unroll
-            for (int d = 0; d < 3; ++d) out[d] = y[d];
+            const bool ov = k > 0 && j < o;
+            place_beads<G>(stile + kl * kTileLd + 3 * j,
+                           kl > 0 ? stile + (kl - 1) * kTileLd + 3 * (s + j) : sprev + 3 * j, smaps + kl,
+                           smaps + (kl > 0 ? kl - 1 : kChunk), ov, dst + ((int64_t)k * s + j) * 3);
         }
         __syncthreads();
         // the chunk's last tile is the next chunk's tile before it
@@ -377,8 +517,11 @@ cudaError_t launch_stitch(const float *coords, const Tiling &t, float *chain, fl
     if (pairs > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const int o = t.T > 1 ? t.overlap : 0;
     const size_t smem = sizeof(float) * kStitchSmemFloats;
-    static_assert(kMapsFloats % 4 == 0, "16-byte alignment of the staged maps");
-    stitch_kernel<<<(unsigned)pairs, kStitchThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
+    static_assert(kMapsFloats % 4 == 0 && kTileLd % 4 == 0, "16-byte alignment of the staged maps and tiles");
+    if (o % 4 == 0)
+        stitch_kernel<4><<<(unsigned)pairs, kStitchThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
+    else
+        stitch_kernel<1><<<(unsigned)pairs, kStitchThreads, smem, st>>>(coords, t.T, t.B, o, chain, resid);
     return cudaGetLastError();
 }
 
