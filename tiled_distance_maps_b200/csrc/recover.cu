@@ -6,9 +6,10 @@
 // x_k = v_k sqrt(max(l_k, 0)).
 //
 // Per map, one warp stages D in shared memory by 16-byte asynchronous copies
-// (the warp's next map is brought into L2 by one bulk prefetch issued when the
-// current map's eigen-solve is done, so those copies wait on L2 rather than
-// DRAM) and forms B = -1/8 J E J from E = (D + D^T)^2 entrywise.  The top
+// and forms B = -1/8 J E J from E = (D + D^T)^2 entrywise.  The copies of the
+// warp's next map go into the same tile as soon as this map's rows are done
+// with: rows 0-31 once the start basis is formed (row l of B is in
+// registers), rows 32-63 once the eigen-solve has converged.  The top
 // eigenpairs come from subspace iteration on three vectors with a
 // Rayleigh-Ritz step (a 3 x 3 Jacobi eigen-solve) every iteration, stopping
 // when the residual of the three Ritz pairs is below kTol * |l_1|.  The start
@@ -204,6 +205,21 @@ __device__ __forceinline__ float sqrt_approx(float x) {
 // three columns of 64 (structure of arrays), and the row means of E.
 constexpr int kWarpFloats = kN * kLd + 3 * kN + kN;
 
+// asynchronous 16-byte copies of rows [32 h, 32 h + 32) of map D into the
+// padded tile, committed as one group
+__device__ __forceinline__ void stage_half(float *sD, const float *D, int h, int lane) {
+    const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(sD));
+#pragma unroll
+    for (int it = 0; it < 16; ++it) {
+        const int idx = it * 32 + lane;
+        const int row = 32 * h + (idx >> 4), c4 = (idx & 15) << 2;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + 4u * (row * kLd + c4)),
+                     "l"(D + row * kN + c4)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
 template <bool DIST>
 __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__restrict__ maps, int64_t n,
                                                                 float *__restrict__ coords,
@@ -217,20 +233,15 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
     float *sR = sV + 3 * kN;       // row means of E, negated
     const int i0 = lane, i1 = lane + 32;
 
-    for (int64_t m = (int64_t)blockIdx.x * kMdsWarps + warp; m < n; m += (int64_t)gridDim.x * kMdsWarps) {
-        const float *D = maps + m * kMapFloats;
-        {   // the map into shared memory by 16-byte asynchronous copies, all in flight at once
-            const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(sE));
-#pragma unroll
-            for (int it = 0; it < 32; ++it) {
-                const int idx = it * 32 + lane;
-                const int row = idx >> 4, c4 = (idx & 15) << 2;
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + 4u * (row * kLd + c4)),
-                             "l"(D + row * kN + c4)
-                             : "memory");
-            }
-            asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
-        }
+    const int64_t stride = (int64_t)gridDim.x * kMdsWarps;
+    int64_t m = (int64_t)blockIdx.x * kMdsWarps + warp;
+    if (m < n) {
+        stage_half(sE, maps + m * kMapFloats, 0, lane);
+        stage_half(sE, maps + m * kMapFloats, 1, lane);
+    }
+    for (; m < n; m += stride) {
+        const int64_t mn = m + stride;    // the warp's next map
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
 
         // e_ij = D_ij + D_ji (twice the symmetric part) and E = e*e, so that
@@ -308,6 +319,12 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                 v0[c] = sE[bi * kLd + i0];     // B[i0][bi] = B[bi][i0]
                 v1[c] = sE[bi * kLd + i1];
             }
+        }
+        // rows 0-31 of B are no longer read (row i0 is in registers): the next
+        // map's first half goes there while this one's eigen-solve runs
+        __syncwarp();
+        if (mn < n) {
+            stage_half(sE, maps + mn * kMapFloats, 0, lane);
         }
         orthonormalize(v0, v1);
 #pragma unroll
@@ -406,15 +423,9 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
                 sV[c * kN + i1] = v1[c];
             }
         }
-        {   // the warp's next map into L2 while this one's coordinates and
-            // distances are written (issued at the start of the map, or before
-            // the eigen-solve, it measured slower)
-            const int64_t mn = m + (int64_t)gridDim.x * kMdsWarps;
-            if (lane == 0 && mn < n)
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(maps + mn * kMapFloats),
-                             "r"((unsigned)(kMapFloats * sizeof(float)))
-                             : "memory");
-        }
+        // rows 32-63 of B are done with too: the next map's second half
+        __syncwarp();
+        if (mn < n) stage_half(sE, maps + mn * kMapFloats, 1, lane);
         if (!conv && lane == 0) atomicOr(flags, (uint32_t)TDM_FLAG_MDS_NOT_CONVERGED);
 
         const float inv_scale = 1.0f / scale;
@@ -434,23 +445,15 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         if (eig != nullptr && lane < 3) eig[m * 3 + lane] = (lane == 0 ? th[0] : lane == 1 ? th[1] : th[2]) * inv_scale;
         if (DIST) {
             // the distance map of the coordinates, as pdist_kernel computes it.
-            // The coordinates go to shared memory twice: as x[64], y[64], z[64]
-            // for the columns (in the V arrays) and, for the rows, as the packed
-            // pairs (x, x, y, y) and (z, z) of each bead (in the E area, free
-            // now).  Lanes 0-15 write row 2p and lanes 16-31 row 2p+1, four
-            // columns per lane, with 16-byte streaming stores.
-            float4 *sb = reinterpret_cast<float4 *>(sE);
-            float2 *sz = reinterpret_cast<float2 *>(sE + 4 * kN);
+            // The coordinates go to shared memory as x[64], y[64], z[64] (in the
+            // V arrays).  Lanes 0-15 write row 2p and lanes 16-31 row 2p+1,
+            // four columns per lane, with 16-byte streaming stores.
             __syncwarp();
 #pragma unroll
             for (int c = 0; c < kK; ++c) {
                 sV[c * kN + i0] = x0[c];
                 sV[c * kN + i1] = x1[c];
             }
-            sb[i0] = make_float4(x0[0], x0[0], x0[1], x0[1]);
-            sb[i1] = make_float4(x1[0], x1[0], x1[1], x1[1]);
-            sz[i0] = make_float2(x0[2], x0[2]);
-            sz[i1] = make_float2(x1[2], x1[2]);
             __syncwarp();
             const int q = lane & 15, h = lane >> 4;
             const float4 cx = ld4(sV + 4 * q), cy = ld4(sV + kN + 4 * q), cz = ld4(sV + 2 * kN + 4 * q);
@@ -461,9 +464,8 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
 #pragma unroll 4
             for (int rp = 0; rp < kN / 2; ++rp) {
                 const int row = 2 * rp + h;
-                const float4 bxy = sb[row];
-                const float2 bz = sz[row];
-                const float2 xx = make_float2(bxy.x, bxy.y), yy = make_float2(bxy.z, bxy.w);
+                const float bx = sV[row], by = sV[kN + row], bzs = sV[2 * kN + row];
+                const float2 xx = make_float2(bx, bx), yy = make_float2(by, by), bz = make_float2(bzs, bzs);
                 const float2 dx01 = __fadd2_rn(xx, nx01), dx23 = __fadd2_rn(xx, nx23);
                 const float2 dy01 = __fadd2_rn(yy, ny01), dy23 = __fadd2_rn(yy, ny23);
                 const float2 dz01 = __fadd2_rn(bz, nz01), dz23 = __fadd2_rn(bz, nz23);
