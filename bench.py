@@ -77,6 +77,7 @@ RUN_SOURCES = ["tiled_distance_maps_b200/csrc/sampler.cu", "tiled_distance_maps_
 REFINE_SOURCES = ["tiled_distance_maps_b200/csrc/refine.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
 DRIFT_SOURCES = ["tiled_distance_maps_b200/csrc/drift.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
 STITCH_SOURCES = ["tiled_distance_maps_b200/csrc/stitch.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
+MDS_SOURCES = ["tiled_distance_maps_b200/csrc/recover.cu", "tiled_distance_maps_b200/csrc/common.cuh"]
 
 
 def profiled_traffic(summary: str, sources) -> int | None:
@@ -107,7 +108,8 @@ def profiled_pipes(summary: str, sources) -> dict | None:
     if profiled_traffic(summary, sources) is None:
         return None
     text = open(os.path.join(ROOT, "profiles", summary)).read()
-    pipes = {m.group(1): float(m.group(2)) / 100.0 for m in re.finditer(r"pipe_(\w+)_pct: ([0-9.]+)", text)}
+    pipes = {m.group(1): float(m.group(2)) / 100.0
+             for m in re.finditer(r"(pipe_\w+|issue_active)_pct: ([0-9.]+)", text)}
     if not pipes:
         return None
     pipes["source"] = f"profiles/{summary} (ncu, one launch of this kernel on this workload)"
@@ -691,6 +693,7 @@ def _mds_rows(nx, n_maps, hbm_gbs):
                      "bound": "hbm", "ms_per_launch": ms, "bytes_per_launch": nbytes,
                      "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm_gbs, "unit": "GB/s",
                      "frac": nbytes / (ms / 1e3) / 1e9 / hbm_gbs, "note": f"{n_maps} maps: {what}"}
+    out["mds_reconstruct"]["traffic"] = profiled_traffic("mds_kernel_chain32_b1000_cfg.md", MDS_SOURCES)
     out["timing"] = "each call timed alone by CUDA events after a 256 MiB write that flushes L2 (median of 10)"
     return out
 
