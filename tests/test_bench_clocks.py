@@ -42,3 +42,24 @@ def test_throttle_reasons_are_reported():
 def test_no_lines_is_reported_as_not_sampled():
     cs = _sampler([], t0=1.0, t1=2.0)
     assert cs.summary()["reasons"] == ["not sampled"]
+
+
+def test_profile_records_are_read_only_for_the_profiled_sources(tmp_path, monkeypatch):
+    # traffic and pipe utilisation come from a committed ncu summary only while
+    # the kernel's sources hash to the value recorded with it
+    import hashlib
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("kernel source\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "k.md").write_text(f"source_sha256: {sha}\ndram_bytes_per_launch: 1234\n"
+                               "    pipe_fma_heavy_pct: 74.3\n    issue_active_pct: 65.2\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("k.md", ["k.cu"]) == 1234
+    pipes = bench.profiled_pipes("k.md", ["k.cu"])
+    assert pipes["pipe_fma_heavy"] == 0.743 and pipes["issue_active"] == 0.652
+    src.write_text("changed\n")
+    assert bench.profiled_traffic("k.md", ["k.cu"]) is None
+    assert bench.profiled_pipes("k.md", ["k.cu"]) is None

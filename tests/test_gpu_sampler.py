@@ -379,3 +379,40 @@ def test_large_and_small_launch_shapes_agree(tdm):
                       return_trajectory=True)
     assert_maps_close(_as5(big, t_big), ref, TOL_MAP, "large launch, final maps")
     assert_maps_close(_as5(part, t_big), traj[S - 2], TOL_MAP, "large launch, state before the last step")
+
+
+def test_compute_entry_points_take_no_device_memory_for_new_shapes(tdm):
+    # The library allocates only when a context or a schedule is created: the
+    # fused run derives its lane map in the kernel, so a new (T, overlap)
+    # shape, a per-step call with the projection and a long stitched chain
+    # leave the free device memory where it was.  Each kernel variant runs
+    # once first (CUDA may load its code lazily on the first launch), and
+    # every buffer is allocated before the first reading.
+    ctx = tdm.context(0)
+    sch = tdm.Schedule(5, ctx=ctx)
+    shapes = ((4, 12), (40, 12), (7, 8), (33, 32), (2, 4))
+    x0s = {(T, o): dev(synth.chain_x0(2, 1, T, overlap=o)).reshape(-1) for T, o in shapes}
+    maps = torch.empty(40 * 3 * 4096, device="cuda")
+    eps = torch.zeros_like(maps)
+    coords = torch.empty(40 * 3 * 192, device="cuda")
+    chain = torch.empty(3 * (64 + 39 * 52) * 3, device="cuda")
+    resid = torch.empty(3 * 39, device="cuda")
+
+    def calls(T, o):
+        t = tdm.Tiling(C=1, T=T, B=3, overlap=o, sync_every=1)
+        n = t.n_maps
+        tdm.ddim_run(sch, maps[:n * 4096], x0s[(T, o)], 1.0, 0.1, 0.3, 5, t, ctx=ctx)
+        tdm.ddim_step(sch, 0, maps[:n * 4096], eps[:n * 4096], eps[:n * 4096], 1.0, 5, t, ctx=ctx)
+        tdm.mds_recover(maps[:n * 4096], n, coords[:n * 192], ctx=ctx)
+        tdm.kabsch_stitch(coords[:n * 192], t, chain[:3 * (64 + (T - 1) * (64 - o)) * 3], resid[:3 * (T - 1)],
+                          ctx=ctx)
+
+    calls(*shapes[0])
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for T, o in shapes[1:]:
+        calls(T, o)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+    assert tdm.ctx_sync(ctx) == 0
