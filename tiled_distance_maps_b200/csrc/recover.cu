@@ -45,28 +45,46 @@ __device__ __forceinline__ float rsqrt_approx(float x) {
     asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
 
 // Gram-Schmidt applied twice per column ("twice is enough") on 64 x kK
-// columns held as rows (l, l+32) per lane.
+// columns held as rows (l, l+32) per lane, in the classical form with the
+// dot products of a round reduced together: four rounds of warp reductions
+// instead of one per dot product.  Round 1 projects a_0 out of a_1 and a_2;
+// round 2 projects it out again and a_1 out of a_2; round 3 projects both
+// out of a_2 again; round 4 normalises.  A column that vanishes becomes zero.
 __device__ __forceinline__ void orthonormalize(float (&a0)[kK], float (&a1)[kK]) {
-#pragma unroll
-    for (int c = 0; c < kK; ++c) {
-#pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-            float d[kK];
-#pragma unroll
-            for (int p = 0; p < c; ++p) d[p] = wsum(fmaf(a0[p], a0[c], a1[p] * a1[c]));
-#pragma unroll
-            for (int p = 0; p < c; ++p) {
-                a0[c] = fmaf(-d[p], a0[p], a0[c]);
-                a1[c] = fmaf(-d[p], a1[p], a1[c]);
-            }
-        }
-        const float nn = wsum(fmaf(a0[c], a0[c], a1[c] * a1[c]));
-        const float inv = nn > 1e-37f ? rsqrt_approx(nn) : 0.0f;
-        a0[c] *= inv;
-        a1[c] *= inv;
-    }
+    const auto dot = [&](int p, int q) { return fmaf(a0[p], a0[q], a1[p] * a1[q]); };
+    const auto axpy = [&](float f, int p, int q) {    // a_q -= f a_p
+        a0[q] = fmaf(-f, a0[p], a0[q]);
+        a1[q] = fmaf(-f, a1[p], a1[q]);
+    };
+    const float g00 = wsum(dot(0, 0)), g01 = wsum(dot(0, 1)), g02 = wsum(dot(0, 2));
+    const float i00 = g00 > 1e-37f ? rcp_approx(g00) : 0.0f;
+    axpy(g01 * i00, 0, 1);
+    axpy(g02 * i00, 0, 2);
+    const float r01 = wsum(dot(0, 1)), r02 = wsum(dot(0, 2)), g11 = wsum(dot(1, 1)), g12 = wsum(dot(1, 2));
+    axpy(r01 * i00, 0, 1);
+    axpy(r02 * i00, 0, 2);
+    const float i11 = g11 > 1e-37f ? rcp_approx(g11) : 0.0f;
+    axpy(g12 * i11, 1, 2);
+    const float p02 = wsum(dot(0, 2)), p12 = wsum(dot(1, 2));
+    axpy(p02 * i00, 0, 2);
+    axpy(p12 * i11, 1, 2);
+    const float n1 = wsum(dot(1, 1)), n2 = wsum(dot(2, 2));
+    const float s0 = g00 > 1e-37f ? rsqrt_approx(g00) : 0.0f;
+    const float s1 = n1 > 1e-37f ? rsqrt_approx(n1) : 0.0f;
+    const float s2 = n2 > 1e-37f ? rsqrt_approx(n2) : 0.0f;
+    a0[0] *= s0;
+    a1[0] *= s0;
+    a0[1] *= s1;
+    a1[1] *= s1;
+    a0[2] *= s2;
+    a1[2] *= s2;
 }
 
 // Orthonormalises the kK columns Y (rows (l, l+32) per lane) whose Gram
@@ -195,11 +213,6 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i) {
     }
 }
 
-__device__ __forceinline__ float sqrt_approx(float x) {
-    float r;
-    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
 
 // Shared memory of one warp: B (the staged D first) at row stride kLd, V as
 // three columns of 64 (structure of arrays), and the row means of E.
@@ -279,7 +292,9 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         // the eigenvalues
         int ex = 0;
         frexpf(gm, &ex);
-        const float scale = gm > 0.0f && isfinite(gm) ? ldexpf(1.0f, -ex) : 1.0f;
+        const bool scaled = gm > 0.0f && isfinite(gm);
+        const float scale = scaled ? ldexpf(1.0f, -ex) : 1.0f;
+        const float inv_scale = scaled ? ldexpf(1.0f, ex) : 1.0f;    // exact: a power of two
         const float cs = -0.125f * scale;
         sR[i0] = -r0;    // negated: a - r is the packed sum a + (-r), rounded as the difference
         sR[i1] = -r1;
@@ -428,11 +443,10 @@ __global__ void __launch_bounds__(kMdsWarps * 32, 3) mds_kernel(const float *__r
         if (mn < n) stage_half(sE, maps + mn * kMapFloats, 1, lane);
         if (!conv && lane == 0) atomicOr(flags, (uint32_t)TDM_FLAG_MDS_NOT_CONVERGED);
 
-        const float inv_scale = 1.0f / scale;
         float x0[kK], x1[kK];
 #pragma unroll
         for (int c = 0; c < kK; ++c) {
-            const float sq = sqrtf(fmaxf(th[c], 0.0f) * inv_scale);
+            const float sq = sqrt_approx(fmaxf(th[c], 0.0f) * inv_scale);
             x0[c] = u0[c] * sq;
             x1[c] = u1[c] * sq;
         }
