@@ -52,10 +52,12 @@ UNIT = "map-steps/s"
 OPS_PHILOX = 40
 OPS_BOX_MULLER_PAIR = 15
 QUADS_PER_MAP = 544
-# SMACOF refinement, per ordered bead pair and Guttman transform: 3 coordinate
-# differences, 3 for the squared distance, 1 reciprocal square root, 1 product
-# with D_ij, 3 accumulating FMAs
-OPS_GUTTMAN_PAIR = 11
+# SMACOF refinement, per unordered bead pair and Guttman transform (each pair
+# is evaluated once and credited to both beads): 3 coordinate differences, 3
+# for the squared distance, 1 reciprocal square root, 1 product with D_ij,
+# 6 accumulating FMAs (3 per bead); 2,016 pairs per map
+OPS_GUTTMAN_PAIR = 14
+GUTTMAN_PAIRS = 64 * 63 // 2
 REFINE_ITERATIONS = 20    # stress within 2e-4 of its 100-iteration value from the MDS start
 SYNC_SWEEP = (0, 1, 2, 5, 10, 25, 50, 3, 7)    # 0 first: the independent run
 
@@ -100,7 +102,17 @@ def profiled_traffic(summary: str, sources) -> int | None:
     return int(nbytes.group(1)) if h.hexdigest()[:16] == sha.group(1) else None
 
 
-def profiled_pipes(summary: str, sources) -> dict | None:
+RUN_PIPES_NOTE = ("the hardware view: fractions of cycles each pipe was busy.  The op-count fraction above counts "
+                  "every Philox round per call (156 lane-ops per quad-step) although the kernel computes round 1 "
+                  "and one product of round 2 once per lane, outside the step loop, and runs the transform and "
+                  "update in packed float32; it is an accounting of the formulation, not a utilisation")
+REFINE_PIPES_NOTE = ("the hardware view: fractions of cycles each pipe was busy.  The kernel evaluates 2,208 pair "
+                     "terms per map-iteration for the 2,016 distinct pairs (offset 8 of the ring and the pairs "
+                     "inside a group are taken by both half-warps at half weight) in packed float32, so the FMA "
+                     "pipe's share is the utilisation")
+
+
+def profiled_pipes(summary: str, sources, note: str = RUN_PIPES_NOTE) -> dict | None:
     """Pipe utilisation of a kernel recorded by an ncu capture in profiles/
     (lines ``pipe_<name>_pct: <value>``), or None when the kernel's sources
     have changed since that capture."""
@@ -113,11 +125,7 @@ def profiled_pipes(summary: str, sources) -> dict | None:
     if not pipes:
         return None
     pipes["source"] = f"profiles/{summary} (ncu, one launch of this kernel on this workload)"
-    pipes["note"] = ("the hardware view: fractions of cycles each pipe was busy.  The op-count fraction above "
-                     "counts every Philox round per call (156 lane-ops per quad-step) although the kernel "
-                     "computes round 1 and one product of round 2 once per lane, outside the step loop, and "
-                     "runs the transform and update in packed float32; it is an accounting of the "
-                     "formulation, not a utilisation")
+    pipes["note"] = note
     return pipes
 
 
@@ -822,7 +830,7 @@ def _workload_records(tdm, ctx, dev, alu_peak, hbm_gbs, pool):
 
 def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs, fma_rate=None):
     """Roofline lines of the kernels beyond the step (rank 0, this GPU)."""
-    ops = n_maps * REFINE_ITERATIONS * 64 * 64 * OPS_GUTTMAN_PAIR
+    ops = n_maps * REFINE_ITERATIONS * GUTTMAN_PAIRS * OPS_GUTTMAN_PAIR
     st_bytes = n_maps * 192 * 4 + B * L * 3 * 4 + B * (T - 1) * 4
     return {
         "timing": "each call timed alone by CUDA events after a 256 MiB write that flushes L2 (median of 10); "
@@ -833,8 +841,10 @@ def _next_rows(nx, n_maps, B, T, L, alu_peak, hbm_gbs, fma_rate=None):
                           "unit": "Tops/s", "frac": ops / (nx["refine_smacof"] / 1e3) / alu_peak,
                           "frac_measured": (ops / (nx["refine_smacof"] / 1e3) / fma_rate) if fma_rate else None,
                           "traffic": profiled_traffic("refine_kernel_chain32_b1000_cfg.md", REFINE_SOURCES),
+                          "pipes": profiled_pipes("refine_kernel_chain32_b1000_cfg.md", REFINE_SOURCES, REFINE_PIPES_NOTE),
                           "note": f"{n_maps} coordinate sets x {REFINE_ITERATIONS} Guttman transforms, "
-                                  f"{OPS_GUTTMAN_PAIR} lane-ops per ordered pair, plus the final stress"},
+                                  f"{OPS_GUTTMAN_PAIR} lane-ops per unordered pair ({GUTTMAN_PAIRS} per map), "
+                                  "plus the final stress (not counted)"},
         "nonoverlap_drift": {"kernel": "drift_sums_kernel", "bound": "hbm", "ms_per_launch": nx["nonoverlap_drift"],
                              "bytes_per_launch": 2 * n_maps * 4096 * 4,
                              "achieved": 2 * n_maps * 4096 * 4 / (nx["nonoverlap_drift"] / 1e3) / 1e9,

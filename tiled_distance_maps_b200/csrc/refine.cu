@@ -7,15 +7,30 @@
 // (x_i - x_j), with d_ij the current distances and terms with d_ij = 0 left
 // out; D is symmetrised first.  A fixed number of iterations is run.
 //
-// Per map, a warp stages D in shared memory with asynchronous copies (issued
-// for the next map while the current one iterates), symmetrises it in place
-// (each unordered pair owned by one lane, so no barrier between reads and
-// writes) and moves rows l and l+32 into registers; lane l then updates beads
-// l and l+32, reading the current coordinates as 128-bit broadcasts from
-// structure-of-arrays copies, four beads per load.  The squared distance of a
-// pair is seeded with FLT_MIN, so a pair at distance zero (the diagonal,
-// coincident beads) contributes w * 0 = 0 without a branch; pairs closer than
-// about 1e-19 are weighted as if that far apart.
+// The pair term w_ij (x_i - x_j), w_ij = D_ij / d_ij, is antisymmetric, so each
+// unordered pair is evaluated once and credited to both beads.  The 64 beads
+// form 16 groups of four (group g = beads 4g..4g+3); lane l of each half-warp
+// owns group l.  Group pairs {g, g+k mod 16} are taken round a ring: the lower
+// half-warp takes offsets k = 1..4, the upper k = 5..8.  At offset k lane l
+// reads group l+k's coordinates (three 128-bit loads from a structure-of-arrays
+// copy), evaluates the 16 bead pairs, adds its own beads' shares to registers
+// and the partner's shares to a travelling accumulator, which moves one lane
+// down the ring before the next offset, so that after the last offset it holds
+// the shares of one group and reaches the owner in one shuffle.  Offset 8 pairs
+// each group pair twice (from both ends) and the pairs inside a group are
+// evaluated by both half-warps, so those weights are halved; the halves' sums
+// are added by one exchange.  Per map-iteration that is 2,208 pair terms
+// (2,016 distinct) against 4,096 when every ordered pair is evaluated.
+//
+// The arithmetic is packed float32: one instruction serves the lane's bead
+// against two partner beads (e = x_partner - x_own, so the own sums are kept
+// negated and the partners' shares need no sign change).  D stays in shared
+// memory only to be read into registers: each lane keeps the 70 symmetrised
+// weights of its pairs, and the copy for the next map is issued while the
+// current one iterates.  The squared distance of a pair is seeded with
+// FLT_MIN, so a pair at distance zero (coincident beads) contributes w * 0 = 0
+// without a branch; pairs closer than about 1e-19 are weighted as if that far
+// apart.
 #include "common.cuh"
 
 namespace tdm {
@@ -24,11 +39,18 @@ namespace {
 constexpr int kRefWarps = 4;
 constexpr int kLdR = kN + 4;
 constexpr int kRefWarpFloats = kN * kLdR + 3 * kN;
+constexpr int kRing = 4;    // ring offsets per half-warp
 constexpr float kQSeed = 1.17549435e-38f;    // FLT_MIN
 
 __device__ __forceinline__ float rsqrt_approx(float x) {
     float r;
     asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
 
@@ -48,154 +70,256 @@ __device__ __forceinline__ void stage_map_async(float *sD, const float *D, int l
 
 __device__ __forceinline__ void wait_staged() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// one pair term: accumulates w (x_i - x_j), w = D_ij / |x_i - x_j|
-__device__ __forceinline__ void guttman_term(float xi, float yi, float zi, float xj, float yj, float zj, float dij,
-                                             float &ax, float &ay, float &az) {
-    const float e0 = xi - xj, e1 = yi - yj, e2 = zi - zj;
-    const float q = fmaf(e2, e2, fmaf(e1, e1, fmaf(e0, e0, kQSeed)));
-    const float w = dij * rsqrt_approx(q);
-    ax = fmaf(w, e0, ax);
-    ay = fmaf(w, e1, ay);
-    az = fmaf(w, e2, az);
+struct Group {    // coordinates of the four beads of one group
+    float x[4], y[4], z[4];
+};
+
+struct Pairs {    // coordinates of a group as float2 pairs: beads (0, 1) and (2, 3)
+    float2 x[2], y[2], z[2];
+};
+
+__device__ __forceinline__ void shuffle_pairs(Pairs &t, int src) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        t.x[c].x = __shfl_sync(0xffffffffu, t.x[c].x, src);
+        t.x[c].y = __shfl_sync(0xffffffffu, t.x[c].y, src);
+        t.y[c].x = __shfl_sync(0xffffffffu, t.y[c].x, src);
+        t.y[c].y = __shfl_sync(0xffffffffu, t.y[c].y, src);
+        t.z[c].x = __shfl_sync(0xffffffffu, t.z[c].x, src);
+        t.z[c].y = __shfl_sync(0xffffffffu, t.z[c].y, src);
+    }
 }
 
-__device__ __forceinline__ float sqrt_approx(float x) {
-    float r;
-    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
+__device__ __forceinline__ Pairs load_pairs(const float *sx, int g) {
+    const float4 px = ld4(sx + 4 * g), py = ld4(sx + kN + 4 * g), pz = ld4(sx + 2 * kN + 4 * g);
+    return Pairs{{make_float2(px.x, px.y), make_float2(px.z, px.w)},
+                 {make_float2(py.x, py.y), make_float2(py.z, py.w)},
+                 {make_float2(pz.x, pz.y), make_float2(pz.z, pz.w)}};
 }
 
-__device__ __forceinline__ float stress_term(float xi, float yi, float zi, float xj, float yj, float zj, float dij) {
-    const float e0 = xi - xj, e1 = yi - yj, e2 = zi - zj;
+// own bead a against partner beads (2cp, 2cp+1) in packed float32: with
+// e = x_partner - x_own, w e is added to the own bead's negated sum and to the
+// partners' shares
+__device__ __forceinline__ void pair_term2(const float2 &nbx, const float2 &nby, const float2 &nbz, const Pairs &p,
+                                           int cp, float2 dij, float2 &ax, float2 &ay, float2 &az, Pairs &t) {
+    const float2 e0 = __fadd2_rn(p.x[cp], nbx), e1 = __fadd2_rn(p.y[cp], nby), e2 = __fadd2_rn(p.z[cp], nbz);
+    float2 q = __ffma2_rn(e0, e0, make_float2(kQSeed, kQSeed));
+    q = __ffma2_rn(e1, e1, q);
+    q = __ffma2_rn(e2, e2, q);
+    const float2 w = __fmul2_rn(dij, make_float2(rsqrt_approx(q.x), rsqrt_approx(q.y)));
+    ax = __ffma2_rn(w, e0, ax);
+    ay = __ffma2_rn(w, e1, ay);
+    az = __ffma2_rn(w, e2, az);
+    t.x[cp] = __ffma2_rn(w, e0, t.x[cp]);
+    t.y[cp] = __ffma2_rn(w, e1, t.y[cp]);
+    t.z[cp] = __ffma2_rn(w, e2, t.z[cp]);
+}
+
+__device__ __forceinline__ float stress_term(const Group &b, int a, const Group &p, int c, float dij) {
+    const float e0 = b.x[a] - p.x[c], e1 = b.y[a] - p.y[c], e2 = b.z[a] - p.z[c];
     const float r = sqrt_approx(fmaf(e2, e2, fmaf(e1, e1, e0 * e0))) - dij;
     return r * r;
 }
 
-struct Beads {    // beads l and l+32 of one lane
-    float x0, y0, z0, x1, y1, z1;
-};
+// index of pair (a, c), a < c, among the six pairs inside a group
+__host__ __device__ constexpr int inner_pair(int a, int c) { return a == 0 ? c - 1 : a == 1 ? c + 1 : 5; }
 
-__device__ __forceinline__ void publish(float *sx, int lane, const Beads &b) {
-    __syncwarp();
-    sx[lane] = b.x0;
-    sx[kN + lane] = b.y0;
-    sx[2 * kN + lane] = b.z0;
-    sx[lane + 32] = b.x1;
-    sx[kN + lane + 32] = b.y1;
-    sx[2 * kN + lane + 32] = b.z1;
-    __syncwarp();
-}
 
-__global__ void __launch_bounds__(kRefWarps * 32) refine_kernel(const float *__restrict__ maps, int64_t n,
-                                                                float *__restrict__ coords, int iterations,
-                                                                float *__restrict__ stress_out) {
+__global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *__restrict__ maps, int64_t n,
+                                                                   float *__restrict__ coords, int iterations,
+                                                                   float *__restrict__ stress_out) {
     extern __shared__ __align__(16) float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = lane >> 4, l = lane & 15;
     float *sD = smem + warp * kRefWarpFloats;
     float *sx = sD + kN * kLdR;    // x[64], y[64], z[64]
     const int64_t stride = (int64_t)gridDim.x * kRefWarps;
     constexpr float kInvN = 1.0f / kN;
+    const int k0 = 1 + kRing * h;                       // first ring offset of this half
+    const int next = (h << 4) | ((l + 1) & 15);          // ring neighbour the accumulator comes from
+    const int owner_src = (h << 4) | ((l - kRing + 1 - k0 + 32) & 15);    // lane holding this group's shares
 
     int64_t m = (int64_t)blockIdx.x * kRefWarps + warp;
     if (m < n) stage_map_async(sD, maps + m * kMapFloats, lane);
     for (; m < n; m += stride) {
         wait_staged();
         __syncwarp();
-        // symmetrise: virtual lane v in {l, l+32} owns the pairs {v, v+k mod 64},
-        // k = 0..32 (k = 32 only for v < 32); every element is read and written
-        // by its owner only, so a batch of offsets can be loaded before it is stored
-#pragma unroll 1
-        for (int k0 = 0; k0 < 32; k0 += 4) {
-            float e[2][4];
+        // symmetrised weights of this lane's pairs; offset 8 (upper half, last
+        // offset) and the pairs inside the group are evaluated twice, at half weight
+        float2 d[kRing][4][2];
+        float dw[6];
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+        for (int s = 0; s < kRing; ++s) {
+            const int g = (l + k0 + s) & 15;
+            const float sc = (h == 1 && s == kRing - 1) ? 0.25f : 0.5f;
+            float4 r[4], t[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int v = lane + 32 * h, w = (v + k0 + u) & (kN - 1);
-                    e[h][u] = 0.5f * (sD[v * kLdR + w] + sD[w * kLdR + v]);
-                }
+            for (int a = 0; a < 4; ++a) {
+                r[a] = ld4(sD + (4 * l + a) * kLdR + 4 * g);
+                t[a] = ld4(sD + (4 * g + a) * kLdR + 4 * l);
+            }
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int v = lane + 32 * h, w = (v + k0 + u) & (kN - 1);
-                    sD[v * kLdR + w] = e[h][u];
-                    sD[w * kLdR + v] = e[h][u];
-                }
+                for (int cp = 0; cp < 2; ++cp)
+                    d[s][a][cp] = make_float2(sc * (comp(r[a], 2 * cp) + comp(t[2 * cp], a)),
+                                              sc * (comp(r[a], 2 * cp + 1) + comp(t[2 * cp + 1], a)));
         }
         {
-            const int w = (lane + 32) & (kN - 1);
-            const float e = 0.5f * (sD[lane * kLdR + w] + sD[w * kLdR + lane]);
-            sD[lane * kLdR + w] = e;
-            sD[w * kLdR + lane] = e;
-        }
-        __syncwarp();
-        float d0[kN], d1[kN];
+            float4 r[4];
 #pragma unroll
-        for (int j4 = 0; j4 < kN / 4; ++j4) {
-            const float4 a = *reinterpret_cast<const float4 *>(sD + lane * kLdR + 4 * j4);
-            const float4 b = *reinterpret_cast<const float4 *>(sD + (lane + 32) * kLdR + 4 * j4);
-            d0[4 * j4] = a.x;
-            d0[4 * j4 + 1] = a.y;
-            d0[4 * j4 + 2] = a.z;
-            d0[4 * j4 + 3] = a.w;
-            d1[4 * j4] = b.x;
-            d1[4 * j4 + 1] = b.y;
-            d1[4 * j4 + 2] = b.z;
-            d1[4 * j4 + 3] = b.w;
+            for (int a = 0; a < 4; ++a) r[a] = ld4(sD + (4 * l + a) * kLdR + 4 * l);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = a + 1; c < 4; ++c) dw[inner_pair(a, c)] = 0.25f * (comp(r[a], c) + comp(r[c], a));
         }
         __syncwarp();
         if (m + stride < n) stage_map_async(sD, maps + (m + stride) * kMapFloats, lane);
 
-        float *X = coords + m * (kN * 3);
-        Beads b{X[3 * lane], X[3 * lane + 1], X[3 * lane + 2],
-                X[3 * (lane + 32)], X[3 * (lane + 32) + 1], X[3 * (lane + 32) + 2]};
-        for (int it = 0; it < iterations; ++it) {
-            publish(sx, lane, b);
-            float a0x = 0.f, a0y = 0.f, a0z = 0.f, a1x = 0.f, a1y = 0.f, a1z = 0.f;
+        float *X = coords + m * (kN * 3) + 12 * l;
+        Group b;
 #pragma unroll
-            for (int j4 = 0; j4 < kN / 4; ++j4) {
-                const float4 px = *reinterpret_cast<const float4 *>(sx + 4 * j4);
-                const float4 py = *reinterpret_cast<const float4 *>(sx + kN + 4 * j4);
-                const float4 pz = *reinterpret_cast<const float4 *>(sx + 2 * kN + 4 * j4);
-                const float jx[4] = {px.x, px.y, px.z, px.w};
-                const float jy[4] = {py.x, py.y, py.z, py.w};
-                const float jz[4] = {pz.x, pz.y, pz.z, pz.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    guttman_term(b.x0, b.y0, b.z0, jx[u], jy[u], jz[u], d0[4 * j4 + u], a0x, a0y, a0z);
-                    guttman_term(b.x1, b.y1, b.z1, jx[u], jy[u], jz[u], d1[4 * j4 + u], a1x, a1y, a1z);
-                }
-            }
-            b = Beads{a0x * kInvN, a0y * kInvN, a0z * kInvN, a1x * kInvN, a1y * kInvN, a1z * kInvN};
+        for (int a = 0; a < 4; ++a) {
+            b.x[a] = X[3 * a];
+            b.y[a] = X[3 * a + 1];
+            b.z[a] = X[3 * a + 2];
         }
-        X[3 * lane] = b.x0;
-        X[3 * lane + 1] = b.y0;
-        X[3 * lane + 2] = b.z0;
-        X[3 * (lane + 32)] = b.x1;
-        X[3 * (lane + 32) + 1] = b.y1;
-        X[3 * (lane + 32) + 2] = b.z1;
-        if (stress_out != nullptr) {
-            publish(sx, lane, b);
-            float acc0 = 0.0f, acc1 = 0.0f;
-#pragma unroll
-            for (int j4 = 0; j4 < kN / 4; ++j4) {
-                const float4 px = *reinterpret_cast<const float4 *>(sx + 4 * j4);
-                const float4 py = *reinterpret_cast<const float4 *>(sx + kN + 4 * j4);
-                const float4 pz = *reinterpret_cast<const float4 *>(sx + 2 * kN + 4 * j4);
-                const float jx[4] = {px.x, px.y, px.z, px.w};
-                const float jy[4] = {py.x, py.y, py.z, py.w};
-                const float jz[4] = {pz.x, pz.y, pz.z, pz.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    acc0 += stress_term(b.x0, b.y0, b.z0, jx[u], jy[u], jz[u], d0[4 * j4 + u]);
-                    acc1 += stress_term(b.x1, b.y1, b.z1, jx[u], jy[u], jz[u], d1[4 * j4 + u]);
-                }
+        for (int it = 0; it < iterations; ++it) {
+            __syncwarp();
+            if (h == 0) {
+                st4(sx + 4 * l, make_float4(b.x[0], b.x[1], b.x[2], b.x[3]));
+                st4(sx + kN + 4 * l, make_float4(b.y[0], b.y[1], b.y[2], b.y[3]));
+                st4(sx + 2 * kN + 4 * l, make_float4(b.z[0], b.z[1], b.z[2], b.z[3]));
             }
-            float acc = acc0 + acc1;
+            __syncwarp();
+            float nx[4], ny[4], nz[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                nx[a] = -b.x[a];
+                ny[a] = -b.y[a];
+                nz[a] = -b.z[a];
+            }
+            float2 ax[4], ay[4], az[4];
+            Pairs t;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) ax[a] = ay[a] = az[a] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) t.x[c] = t.y[c] = t.z[c] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int s = 0; s < kRing; ++s) {
+                const Pairs p = load_pairs(sx, (l + k0 + s) & 15);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int cp = 0; cp < 2; ++cp)
+                        pair_term2(make_float2(nx[a], nx[a]), make_float2(ny[a], ny[a]), make_float2(nz[a], nz[a]),
+                                   p, cp, d[s][a][cp], ax[a], ay[a], az[a], t);
+                if (s + 1 < kRing) shuffle_pairs(t, next);
+            }
+            // own sums (negated), pairs inside the group, then the partners' shares
+            float sx_[4], sy_[4], sz_[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                sx_[a] = ax[a].x + ax[a].y;
+                sy_[a] = ay[a].x + ay[a].y;
+                sz_[a] = az[a].x + az[a].y;
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = a + 1; c < 4; ++c) {
+                    const float e0 = nx[a] - nx[c], e1 = ny[a] - ny[c], e2 = nz[a] - nz[c];
+                    const float q = fmaf(e2, e2, fmaf(e1, e1, fmaf(e0, e0, kQSeed)));
+                    const float w = dw[inner_pair(a, c)] * rsqrt_approx(q);
+                    sx_[a] = fmaf(w, e0, sx_[a]);
+                    sy_[a] = fmaf(w, e1, sy_[a]);
+                    sz_[a] = fmaf(w, e2, sz_[a]);
+                    sx_[c] = fmaf(-w, e0, sx_[c]);
+                    sy_[c] = fmaf(-w, e1, sy_[c]);
+                    sz_[c] = fmaf(-w, e2, sz_[c]);
+                }
+            shuffle_pairs(t, owner_src);
+            float tx[4] = {t.x[0].x, t.x[0].y, t.x[1].x, t.x[1].y};
+            float ty[4] = {t.y[0].x, t.y[0].y, t.y[1].x, t.y[1].y};
+            float tz[4] = {t.z[0].x, t.z[0].y, t.z[1].x, t.z[1].y};
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                tx[a] -= sx_[a];
+                ty[a] -= sy_[a];
+                tz[a] -= sz_[a];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                tx[a] += __shfl_xor_sync(0xffffffffu, tx[a], 16);
+                ty[a] += __shfl_xor_sync(0xffffffffu, ty[a], 16);
+                tz[a] += __shfl_xor_sync(0xffffffffu, tz[a], 16);
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                b.x[a] = tx[a] * kInvN;
+                b.y[a] = ty[a] * kInvN;
+                b.z[a] = tz[a] * kInvN;
+            }
+        }
+        if (h == 0) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                X[3 * a] = b.x[a];
+                X[3 * a + 1] = b.y[a];
+                X[3 * a + 2] = b.z[a];
+            }
+        }
+        if (stress_out != nullptr) {
+            __syncwarp();
+            if (h == 0) {
+                st4(sx + 4 * l, make_float4(b.x[0], b.x[1], b.x[2], b.x[3]));
+                st4(sx + kN + 4 * l, make_float4(b.y[0], b.y[1], b.y[2], b.y[3]));
+                st4(sx + 2 * kN + 4 * l, make_float4(b.z[0], b.z[1], b.z[2], b.z[3]));
+            }
+            __syncwarp();
+            // every unordered pair once: the weights halved above are doubled
+            // back and their terms counted at half weight
+            float nx[4], ny[4], nz[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                nx[a] = -b.x[a];
+                ny[a] = -b.y[a];
+                nz[a] = -b.z[a];
+            }
+            float2 acc2 = make_float2(0.0f, 0.0f), last2 = make_float2(0.0f, 0.0f);
+            const float2 m1 = make_float2(-1.0f, -1.0f);
+            const float2 up = h == 1 ? make_float2(2.0f, 2.0f) : make_float2(1.0f, 1.0f);
+#pragma unroll
+            for (int s = 0; s < kRing; ++s) {
+                const Pairs p = load_pairs(sx, (l + k0 + s) & 15);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int cp = 0; cp < 2; ++cp) {
+                        const float2 e0 = __fadd2_rn(p.x[cp], make_float2(nx[a], nx[a]));
+                        const float2 e1 = __fadd2_rn(p.y[cp], make_float2(ny[a], ny[a]));
+                        const float2 e2 = __fadd2_rn(p.z[cp], make_float2(nz[a], nz[a]));
+                        float2 q = __fmul2_rn(e0, e0);
+                        q = __ffma2_rn(e1, e1, q);
+                        q = __ffma2_rn(e2, e2, q);
+                        const float2 dd = s == kRing - 1 ? __fmul2_rn(d[s][a][cp], up) : d[s][a][cp];
+                        const float2 r = __ffma2_rn(dd, m1, make_float2(sqrt_approx(q.x), sqrt_approx(q.y)));
+                        if (s == kRing - 1) last2 = __ffma2_rn(r, r, last2);
+                        else acc2 = __ffma2_rn(r, r, acc2);
+                    }
+            }
+            float twice = 0.0f;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int c = a + 1; c < 4; ++c) twice += stress_term(b, a, b, c, 2.0f * dw[inner_pair(a, c)]);
+            // the last offset's terms count at half weight in the upper half (offset 8)
+            float acc = fmaf(h == 1 ? 0.5f : 1.0f, last2.x + last2.y, acc2.x + acc2.y);
+            acc = fmaf(0.5f, twice, acc);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (lane == 0) stress_out[m] = 0.5f * acc;    // each unordered pair appears twice
+            if (lane == 0) stress_out[m] = acc;
         }
     }
 }
