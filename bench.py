@@ -106,10 +106,10 @@ RUN_PIPES_NOTE = ("the hardware view: fractions of cycles each pipe was busy.  T
                   "every Philox round per call (156 lane-ops per quad-step) although the kernel computes round 1 "
                   "and one product of round 2 once per lane, outside the step loop, and runs the transform and "
                   "update in packed float32; it is an accounting of the formulation, not a utilisation")
-REFINE_PIPES_NOTE = ("the hardware view: fractions of cycles each pipe was busy.  The kernel evaluates 2,208 pair "
-                     "terms per map-iteration for the 2,016 distinct pairs (offset 8 of the ring and the pairs "
-                     "inside a group are taken by both half-warps at half weight) in packed float32, so the FMA "
-                     "pipe's share is the utilisation")
+REFINE_PIPES_NOTE = ("the hardware view: fractions of cycles each pipe was busy.  The kernel evaluates 2,144 pair "
+                     "terms per map-iteration for the 2,016 distinct pairs (offset 8 of the ring is taken by both "
+                     "half-warps at half weight) in packed float32, so the FMA pipe's share is the utilisation; the "
+                     "packed pair term alone keeps that pipe at most 84 % busy")
 
 
 def profiled_pipes(summary: str, sources, note: str = RUN_PIPES_NOTE) -> dict | None:

@@ -16,15 +16,18 @@
 // copy), evaluates the 16 bead pairs, adds its own beads' shares to registers
 // and the partner's shares to a travelling accumulator, which moves one lane
 // down the ring before the next offset, so that after the last offset it holds
-// the shares of one group and reaches the owner in one shuffle.  Offset 8 pairs
-// each group pair twice (from both ends) and the pairs inside a group are
-// evaluated by both half-warps, so those weights are halved; the halves' sums
-// are added by one exchange.  Per map-iteration that is 2,208 pair terms
-// (2,016 distinct) against 4,096 when every ordered pair is evaluated.
+// the shares of one group and reaches the owner in one shuffle.  Offset 8 meets
+// each group pair from both ends, so its weights are halved.  Of the six pairs
+// inside a group each half-warp takes three: the upper half holds its beads in
+// a rotated register order, so the same register pairs name other bead pairs.
+// The halves' sums are added by one exchange.  Per map-iteration that is 2,144
+// pair terms (2,016 distinct) against 4,096 when every ordered pair is
+// evaluated.
 //
 // The arithmetic is packed float32: one instruction serves the lane's bead
-// against two partner beads (e = x_partner - x_own, so the own sums are kept
-// negated and the partners' shares need no sign change).  D stays in shared
+// against two partner beads (e = x_partner - x_own, formed as an FMA with -1,
+// so the own sums are kept negated and the partners' shares need no sign
+// change).  D stays in shared
 // memory only to be read into registers: each lane keeps the 70 symmetrised
 // weights of its pairs, and the copy for the next map is issued while the
 // current one iterates.  The squared distance of a pair is seeded with
@@ -97,12 +100,14 @@ __device__ __forceinline__ Pairs load_pairs(const float *sx, int g) {
                  {make_float2(pz.x, pz.y), make_float2(pz.z, pz.w)}};
 }
 
-// own bead a against partner beads (2cp, 2cp+1) in packed float32: with
-// e = x_partner - x_own, w e is added to the own bead's negated sum and to the
-// partners' shares
-__device__ __forceinline__ void pair_term2(const float2 &nbx, const float2 &nby, const float2 &nbz, const Pairs &p,
+// own bead (bx, by, bz), broadcast, against partner beads (2cp, 2cp+1) in
+// packed float32: with e = x_partner - x_own, w e is added to the own bead's
+// negated sum and to the partners' shares
+__device__ __forceinline__ void pair_term2(const float2 &bx, const float2 &by, const float2 &bz, const Pairs &p,
                                            int cp, float2 dij, float2 &ax, float2 &ay, float2 &az, Pairs &t) {
-    const float2 e0 = __fadd2_rn(p.x[cp], nbx), e1 = __fadd2_rn(p.y[cp], nby), e2 = __fadd2_rn(p.z[cp], nbz);
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+    const float2 e0 = __ffma2_rn(bx, m1, p.x[cp]), e1 = __ffma2_rn(by, m1, p.y[cp]),
+                 e2 = __ffma2_rn(bz, m1, p.z[cp]);
     float2 q = __ffma2_rn(e0, e0, make_float2(kQSeed, kQSeed));
     q = __ffma2_rn(e1, e1, q);
     q = __ffma2_rn(e2, e2, q);
@@ -115,14 +120,27 @@ __device__ __forceinline__ void pair_term2(const float2 &nbx, const float2 &nby,
     t.z[cp] = __ffma2_rn(w, e2, t.z[cp]);
 }
 
+// Register order of the own beads: the lower half-warp keeps beads 0..3 in
+// registers 0..3, the upper half-warp bead (a + 3) mod 4 in register a.  Then
+// the same three register pairs (0, 1), (2, 3), (0, 2) are the bead pairs
+// (0,1), (2,3), (0,2) in one half and (3,0), (1,2), (3,1) in the other: the
+// six pairs inside a group, each once.
+__device__ __forceinline__ int bead_of(int h, int a) { return h ? (a + 3) & 3 : a; }
+// hi where sel = 0x7654, lo where sel = 0x3210: a byte permute, so that the
+// choice between two registers is never turned into an indexed access
+__device__ __forceinline__ float pick(unsigned sel, float hi, float lo) {
+    return __int_as_float((int)__byte_perm((unsigned)__float_as_int(lo), (unsigned)__float_as_int(hi), sel));
+}
+__device__ __forceinline__ float rot(unsigned up, const float (&v)[4], int a) { return pick(up, v[(a + 3) & 3], v[a]); }
+__device__ __forceinline__ float unrot(unsigned up, const float (&v)[4], int a) { return pick(up, v[(a + 1) & 3], v[a]); }
+__host__ __device__ constexpr int inner_u(int j) { return j == 1 ? 2 : 0; }
+__host__ __device__ constexpr int inner_v(int j) { return j == 0 ? 1 : j == 1 ? 3 : 2; }
+
 __device__ __forceinline__ float stress_term(const Group &b, int a, const Group &p, int c, float dij) {
     const float e0 = b.x[a] - p.x[c], e1 = b.y[a] - p.y[c], e2 = b.z[a] - p.z[c];
     const float r = sqrt_approx(fmaf(e2, e2, fmaf(e1, e1, e0 * e0))) - dij;
     return r * r;
 }
-
-// index of pair (a, c), a < c, among the six pairs inside a group
-__host__ __device__ constexpr int inner_pair(int a, int c) { return a == 0 ? c - 1 : a == 1 ? c + 1 : 5; }
 
 
 __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *__restrict__ maps, int64_t n,
@@ -139,24 +157,33 @@ __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *
     const int next = (h << 4) | ((l + 1) & 15);          // ring neighbour the accumulator comes from
     const int owner_src = (h << 4) | ((l - kRing + 1 - k0 + 32) & 15);    // lane holding this group's shares
 
+    const bool up = h == 1;
+    const unsigned sel = up ? 0x7654u : 0x3210u;    // byte-permute selector of the upper half
+
     int64_t m = (int64_t)blockIdx.x * kRefWarps + warp;
     if (m < n) stage_map_async(sD, maps + m * kMapFloats, lane);
     for (; m < n; m += stride) {
         wait_staged();
         __syncwarp();
-        // symmetrised weights of this lane's pairs; offset 8 (upper half, last
-        // offset) and the pairs inside the group are evaluated twice, at half weight
+        // symmetrised weights of this lane's pairs, own beads in register
+        // order; offset 8 (upper half, last offset) meets each group pair from
+        // both ends, so its weights are halved
         float2 d[kRing][4][2];
-        float dw[6];
+        float dw[3];
 #pragma unroll
         for (int s = 0; s < kRing; ++s) {
             const int g = (l + k0 + s) & 15;
-            const float sc = (h == 1 && s == kRing - 1) ? 0.25f : 0.5f;
+            const float sc = (up && s == kRing - 1) ? 0.25f : 0.5f;
             float4 r[4], t[4];
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
-                r[a] = ld4(sD + (4 * l + a) * kLdR + 4 * g);
+                r[a] = ld4(sD + (4 * l + bead_of(h, a)) * kLdR + 4 * g);
                 t[a] = ld4(sD + (4 * g + a) * kLdR + 4 * l);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float v[4] = {t[c].x, t[c].y, t[c].z, t[c].w};
+                t[c] = make_float4(rot(sel, v, 0), rot(sel, v, 1), rot(sel, v, 2), rot(sel, v, 3));
             }
 #pragma unroll
             for (int a = 0; a < 4; ++a)
@@ -169,16 +196,18 @@ __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *
             float4 r[4];
 #pragma unroll
             for (int a = 0; a < 4; ++a) r[a] = ld4(sD + (4 * l + a) * kLdR + 4 * l);
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = a + 1; c < 4; ++c) dw[inner_pair(a, c)] = 0.25f * (comp(r[a], c) + comp(r[c], a));
+            // register pairs (0,1), (2,3), (0,2): bead pairs (0,1), (2,3), (0,2)
+            // in the lower half, (3,0), (1,2), (3,1) in the upper
+            auto ds = [&](int a, int c) { return 0.5f * (comp(r[a], c) + comp(r[c], a)); };
+            dw[0] = pick(sel, ds(3, 0), ds(0, 1));
+            dw[1] = pick(sel, ds(1, 2), ds(2, 3));
+            dw[2] = pick(sel, ds(3, 1), ds(0, 2));
         }
         __syncwarp();
         if (m + stride < n) stage_map_async(sD, maps + (m + stride) * kMapFloats, lane);
 
         float *X = coords + m * (kN * 3) + 12 * l;
-        Group b;
+        Group b;    // bead order
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
             b.x[a] = X[3 * a];
@@ -193,12 +222,12 @@ __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *
                 st4(sx + 2 * kN + 4 * l, make_float4(b.z[0], b.z[1], b.z[2], b.z[3]));
             }
             __syncwarp();
-            float nx[4], ny[4], nz[4];
+            Group r;    // register order
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
-                nx[a] = -b.x[a];
-                ny[a] = -b.y[a];
-                nz[a] = -b.z[a];
+                r.x[a] = rot(sel, b.x, a);
+                r.y[a] = rot(sel, b.y, a);
+                r.z[a] = rot(sel, b.z, a);
             }
             float2 ax[4], ay[4], az[4];
             Pairs t;
@@ -213,11 +242,12 @@ __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *
                 for (int a = 0; a < 4; ++a)
 #pragma unroll
                     for (int cp = 0; cp < 2; ++cp)
-                        pair_term2(make_float2(nx[a], nx[a]), make_float2(ny[a], ny[a]), make_float2(nz[a], nz[a]),
-                                   p, cp, d[s][a][cp], ax[a], ay[a], az[a], t);
+                        pair_term2(make_float2(r.x[a], r.x[a]), make_float2(r.y[a], r.y[a]),
+                                   make_float2(r.z[a], r.z[a]), p, cp, d[s][a][cp], ax[a], ay[a], az[a], t);
                 if (s + 1 < kRing) shuffle_pairs(t, next);
             }
-            // own sums (negated), pairs inside the group, then the partners' shares
+            // own sums (negated, register order) and this half's three pairs
+            // inside the group
             float sx_[4], sy_[4], sz_[4];
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
@@ -226,28 +256,27 @@ __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *
                 sz_[a] = az[a].x + az[a].y;
             }
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = a + 1; c < 4; ++c) {
-                    const float e0 = nx[a] - nx[c], e1 = ny[a] - ny[c], e2 = nz[a] - nz[c];
-                    const float q = fmaf(e2, e2, fmaf(e1, e1, fmaf(e0, e0, kQSeed)));
-                    const float w = dw[inner_pair(a, c)] * rsqrt_approx(q);
-                    sx_[a] = fmaf(w, e0, sx_[a]);
-                    sy_[a] = fmaf(w, e1, sy_[a]);
-                    sz_[a] = fmaf(w, e2, sz_[a]);
-                    sx_[c] = fmaf(-w, e0, sx_[c]);
-                    sy_[c] = fmaf(-w, e1, sy_[c]);
-                    sz_[c] = fmaf(-w, e2, sz_[c]);
-                }
+            for (int j = 0; j < 3; ++j) {
+                const int u = inner_u(j), v = inner_v(j);
+                const float e0 = r.x[v] - r.x[u], e1 = r.y[v] - r.y[u], e2 = r.z[v] - r.z[u];
+                const float q = fmaf(e2, e2, fmaf(e1, e1, fmaf(e0, e0, kQSeed)));
+                const float w = dw[j] * rsqrt_approx(q);
+                sx_[u] = fmaf(w, e0, sx_[u]);
+                sy_[u] = fmaf(w, e1, sy_[u]);
+                sz_[u] = fmaf(w, e2, sz_[u]);
+                sx_[v] = fmaf(-w, e0, sx_[v]);
+                sy_[v] = fmaf(-w, e1, sy_[v]);
+                sz_[v] = fmaf(-w, e2, sz_[v]);
+            }
             shuffle_pairs(t, owner_src);
             float tx[4] = {t.x[0].x, t.x[0].y, t.x[1].x, t.x[1].y};
             float ty[4] = {t.y[0].x, t.y[0].y, t.y[1].x, t.y[1].y};
             float tz[4] = {t.z[0].x, t.z[0].y, t.z[1].x, t.z[1].y};
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
-                tx[a] -= sx_[a];
-                ty[a] -= sy_[a];
-                tz[a] -= sz_[a];
+                tx[a] -= unrot(sel, sx_, a);
+                ty[a] -= unrot(sel, sy_, a);
+                tz[a] -= unrot(sel, sz_, a);
             }
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
@@ -278,18 +307,18 @@ __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *
                 st4(sx + 2 * kN + 4 * l, make_float4(b.z[0], b.z[1], b.z[2], b.z[3]));
             }
             __syncwarp();
-            // every unordered pair once: the weights halved above are doubled
-            // back and their terms counted at half weight
-            float nx[4], ny[4], nz[4];
+            // every unordered pair once: offset 8's halved weights are doubled
+            // back and its terms counted at half weight
+            Group r;
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
-                nx[a] = -b.x[a];
-                ny[a] = -b.y[a];
-                nz[a] = -b.z[a];
+                r.x[a] = rot(sel, b.x, a);
+                r.y[a] = rot(sel, b.y, a);
+                r.z[a] = rot(sel, b.z, a);
             }
             float2 acc2 = make_float2(0.0f, 0.0f), last2 = make_float2(0.0f, 0.0f);
             const float2 m1 = make_float2(-1.0f, -1.0f);
-            const float2 up = h == 1 ? make_float2(2.0f, 2.0f) : make_float2(1.0f, 1.0f);
+            const float2 dbl = up ? make_float2(2.0f, 2.0f) : make_float2(1.0f, 1.0f);
 #pragma unroll
             for (int s = 0; s < kRing; ++s) {
                 const Pairs p = load_pairs(sx, (l + k0 + s) & 15);
@@ -297,26 +326,21 @@ __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *
                 for (int a = 0; a < 4; ++a)
 #pragma unroll
                     for (int cp = 0; cp < 2; ++cp) {
-                        const float2 e0 = __fadd2_rn(p.x[cp], make_float2(nx[a], nx[a]));
-                        const float2 e1 = __fadd2_rn(p.y[cp], make_float2(ny[a], ny[a]));
-                        const float2 e2 = __fadd2_rn(p.z[cp], make_float2(nz[a], nz[a]));
+                        const float2 e0 = __ffma2_rn(make_float2(r.x[a], r.x[a]), m1, p.x[cp]);
+                        const float2 e1 = __ffma2_rn(make_float2(r.y[a], r.y[a]), m1, p.y[cp]);
+                        const float2 e2 = __ffma2_rn(make_float2(r.z[a], r.z[a]), m1, p.z[cp]);
                         float2 q = __fmul2_rn(e0, e0);
                         q = __ffma2_rn(e1, e1, q);
                         q = __ffma2_rn(e2, e2, q);
-                        const float2 dd = s == kRing - 1 ? __fmul2_rn(d[s][a][cp], up) : d[s][a][cp];
-                        const float2 r = __ffma2_rn(dd, m1, make_float2(sqrt_approx(q.x), sqrt_approx(q.y)));
-                        if (s == kRing - 1) last2 = __ffma2_rn(r, r, last2);
-                        else acc2 = __ffma2_rn(r, r, acc2);
+                        const float2 dd = s == kRing - 1 ? __fmul2_rn(d[s][a][cp], dbl) : d[s][a][cp];
+                        const float2 rr = __ffma2_rn(dd, m1, make_float2(sqrt_approx(q.x), sqrt_approx(q.y)));
+                        if (s == kRing - 1) last2 = __ffma2_rn(rr, rr, last2);
+                        else acc2 = __ffma2_rn(rr, rr, acc2);
                     }
             }
-            float twice = 0.0f;
+            float acc = fmaf(up ? 0.5f : 1.0f, last2.x + last2.y, acc2.x + acc2.y);
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = a + 1; c < 4; ++c) twice += stress_term(b, a, b, c, 2.0f * dw[inner_pair(a, c)]);
-            // the last offset's terms count at half weight in the upper half (offset 8)
-            float acc = fmaf(h == 1 ? 0.5f : 1.0f, last2.x + last2.y, acc2.x + acc2.y);
-            acc = fmaf(0.5f, twice, acc);
+            for (int j = 0; j < 3; ++j) acc += stress_term(r, inner_u(j), r, inner_v(j), dw[j]);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
             if (lane == 0) stress_out[m] = acc;
