@@ -27,13 +27,12 @@
 // The arithmetic is packed float32: one instruction serves the lane's bead
 // against two partner beads (e = x_partner - x_own, formed as an FMA with -1,
 // so the own sums are kept negated and the partners' shares need no sign
-// change).  D stays in shared
-// memory only to be read into registers: each lane keeps the 70 symmetrised
-// weights of its pairs, and the copy for the next map is issued while the
-// current one iterates.  The squared distance of a pair is seeded with
-// FLT_MIN, so a pair at distance zero (coincident beads) contributes w * 0 = 0
-// without a branch; pairs closer than about 1e-19 are weighted as if that far
-// apart.
+// change).  D stays in shared memory only to be read into registers: each lane
+// keeps the 67 symmetrised weights of its pairs, and the copy for the next map
+// is issued while the current one iterates.  The squared distance of a pair is
+// seeded with FLT_MIN, so a pair at distance zero (coincident beads)
+// contributes w * 0 = 0 without a branch; pairs closer than about 1e-19 are
+// weighted as if that far apart.
 #include "common.cuh"
 
 namespace tdm {
@@ -131,8 +130,8 @@ __device__ __forceinline__ int bead_of(int h, int a) { return h ? (a + 3) & 3 : 
 __device__ __forceinline__ float pick(unsigned sel, float hi, float lo) {
     return __int_as_float((int)__byte_perm((unsigned)__float_as_int(lo), (unsigned)__float_as_int(hi), sel));
 }
-__device__ __forceinline__ float rot(unsigned up, const float (&v)[4], int a) { return pick(up, v[(a + 3) & 3], v[a]); }
-__device__ __forceinline__ float unrot(unsigned up, const float (&v)[4], int a) { return pick(up, v[(a + 1) & 3], v[a]); }
+__device__ __forceinline__ float rot(unsigned sel, const float (&v)[4], int a) { return pick(sel, v[(a + 3) & 3], v[a]); }
+__device__ __forceinline__ float unrot(unsigned sel, const float (&v)[4], int a) { return pick(sel, v[(a + 1) & 3], v[a]); }
 __host__ __device__ constexpr int inner_u(int j) { return j == 1 ? 2 : 0; }
 __host__ __device__ constexpr int inner_v(int j) { return j == 0 ? 1 : j == 1 ? 3 : 2; }
 
@@ -141,7 +140,6 @@ __device__ __forceinline__ float stress_term(const Group &b, int a, const Group 
     const float r = sqrt_approx(fmaf(e2, e2, fmaf(e1, e1, e0 * e0))) - dij;
     return r * r;
 }
-
 
 __global__ void __launch_bounds__(kRefWarps * 32, 2) refine_kernel(const float *__restrict__ maps, int64_t n,
                                                                    float *__restrict__ coords, int iterations,
