@@ -108,8 +108,7 @@ RUN_PIPES_NOTE = ("the hardware view: fractions of cycles each pipe was busy.  T
                   "update in packed float32; it is an accounting of the formulation, not a utilisation")
 REFINE_PIPES_NOTE = ("the hardware view: fractions of cycles each pipe was busy.  The kernel evaluates 2,144 pair "
                      "terms per map-iteration for the 2,016 distinct pairs (offset 8 of the ring is taken by both "
-                     "half-warps at half weight) in packed float32, so the FMA pipe's share is the utilisation; the "
-                     "packed pair term alone keeps that pipe at most 84 % busy")
+                     "half-warps at half weight) in packed float32, so the FMA pipe's share is the utilisation")
 
 
 def profiled_pipes(summary: str, sources, note: str = RUN_PIPES_NOTE) -> dict | None:
